@@ -1,0 +1,180 @@
+"""CPU oracle for the NVFP4 W4A16 linear layer (ctypes wrapper of nvfp4_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product library (``gemm_decode_nvfp4_b200``) never imports it and
+has no CPU fallback.
+
+The C file states what each function follows on the pages and the readings
+taken where the pages are silent.  Every function here is pinned by the
+``-m "not gpu"`` tests against facts the format fixes (the sixteen E2M1
+values, E4M3 bit fields, library casts in ml_dtypes, brute force on tiny
+inputs, exact round trips, the shared-scale identity).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB = os.path.join(_HERE, "libnvfp4_oracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (fp32 kept strict: no contraction, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", _LIB + ".tmp", _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        c_i64, c_f, c_p = ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
+        L.oracle_e2m1_decode.argtypes = [ctypes.c_int]
+        L.oracle_e2m1_decode.restype = ctypes.c_double
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_int]
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_rne_satfinite.argtypes = [c_f]
+        L.oracle_e4m3_rne_satfinite.restype = ctypes.c_int
+        L.oracle_e2m1_rne_satfinite.argtypes = [c_f]
+        L.oracle_e2m1_rne_satfinite.restype = ctypes.c_int
+        L.oracle_amax.argtypes = [c_p, c_i64, c_i64, c_i64]
+        L.oracle_amax.restype = c_f
+        L.oracle_tensor_scale.argtypes = [c_f]
+        L.oracle_tensor_scale.restype = c_f
+        L.oracle_quantize.argtypes = [c_p, c_i64, c_i64, c_i64, c_f, c_p, c_p]
+        L.oracle_quantize.restype = None
+        L.oracle_dequantize.argtypes = [c_p, c_p, c_f, c_i64, c_i64, c_p]
+        L.oracle_dequantize.restype = None
+        L.oracle_linear.argtypes = [c_p, c_i64, c_p, c_p, c_f, c_i64, c_i64, c_i64,
+                                    c_p, c_p, c_i64, c_p, c_p]
+        L.oracle_linear.restype = None
+        L.oracle_num_threads.argtypes = []
+        L.oracle_num_threads.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bf16_bits(w) -> np.ndarray:
+    """BF16 torch tensor (or uint16 array) -> contiguous uint16 numpy view."""
+    if isinstance(w, np.ndarray):
+        assert w.dtype == np.uint16
+        return np.ascontiguousarray(w)
+    import torch
+    assert w.dtype == torch.bfloat16
+    return np.ascontiguousarray(w.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+# ----------------------------------------------------------- scalar helpers
+
+def e2m1_decode(code: int) -> float:
+    return lib().oracle_e2m1_decode(int(code))
+
+
+def e4m3_decode(byte: int) -> float:
+    return lib().oracle_e4m3_decode(int(byte))
+
+
+def e4m3_rne_satfinite(v: float) -> int:
+    return lib().oracle_e4m3_rne_satfinite(float(np.float32(v)))
+
+
+def e2m1_rne_satfinite(v: float) -> int:
+    return lib().oracle_e2m1_rne_satfinite(float(np.float32(v)))
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+# ----------------------------------------------------------- tensor helpers
+
+def amax(w) -> np.float32:
+    """max |w| of a BF16 matrix (2-D) or vector."""
+    b = _bf16_bits(w)
+    if b.ndim == 1:
+        b = b.reshape(1, -1)
+    rows, cols = b.shape
+    return np.float32(lib().oracle_amax(_ptr(b), rows, cols, cols))
+
+
+def tensor_scale(a) -> np.float32:
+    """g = amax / (6 * 448) in fp32."""
+    return np.float32(lib().oracle_tensor_scale(float(np.float32(a))))
+
+
+def quantize(w, g=None):
+    """RTN NVFP4 of a BF16 [N, K] matrix.  Returns (q [N, K/2] u8, s [N, K/16] u8,
+    g fp32).  g defaults to this tensor's own amax / 2688; pass the shared g of
+    a merged layer to quantize one member."""
+    b = _bf16_bits(w)
+    N, K = b.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    if g is None:
+        g = tensor_scale(amax(b))
+    g = np.float32(g)
+    q = np.empty((N, K // 2), np.uint8)
+    s = np.empty((N, K // 16), np.uint8)
+    lib().oracle_quantize(_ptr(b), N, K, K, float(g), _ptr(q), _ptr(s))
+    return q, s, g
+
+
+def dequantize(q: np.ndarray, s: np.ndarray, g) -> np.ndarray:
+    """W_deq [N, K] in fp64."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    N, K = q.shape[0], q.shape[1] * 2
+    out = np.empty((N, K), np.float64)
+    lib().oracle_dequantize(_ptr(q), _ptr(s), float(np.float32(g)), N, K, _ptr(out))
+    return out
+
+
+def linear(x, q: np.ndarray, s: np.ndarray, g, rows=None, cols=None):
+    """y = x . W^T in fp64 with the per-element magnitude bound sum |w x|.
+
+    x is BF16 [M, K] (or [K]).  With rows/cols (equal-length index arrays) only
+    those outputs are computed and 1-D arrays are returned; otherwise [M, N]."""
+    xb = _bf16_bits(x)
+    if xb.ndim == 1:
+        xb = xb.reshape(1, -1)
+    M, K = xb.shape
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    N = q.shape[0]
+    assert q.shape[1] * 2 == K and s.shape == (N, K // 16)
+    if rows is None:
+        y = np.empty((M, N), np.float64)
+        bound = np.empty((M, N), np.float64)
+        lib().oracle_linear(_ptr(xb), K, _ptr(q), _ptr(s), float(np.float32(g)), M, N, K,
+                            None, None, -1, _ptr(y), _ptr(bound))
+        return y, bound
+    ri = np.ascontiguousarray(rows, np.int64)
+    ci = np.ascontiguousarray(cols, np.int64)
+    assert ri.shape == ci.shape and ri.ndim == 1
+    y = np.empty(ri.shape, np.float64)
+    bound = np.empty(ri.shape, np.float64)
+    lib().oracle_linear(_ptr(xb), K, _ptr(q), _ptr(s), float(np.float32(g)), M, N, K,
+                        _ptr(ri), _ptr(ci), len(ri), _ptr(y), _ptr(bound))
+    return y, bound
+
+
+def tolerance(y_ref: np.ndarray, bound: np.ndarray) -> np.ndarray:
+    """Acceptance bound per output: 1e-3 * sum|w x| + 1e-2 * |y_ref|."""
+    return 1e-3 * bound + 1e-2 * np.abs(y_ref)
