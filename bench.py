@@ -1,0 +1,452 @@
+"""Benchmark of the NVFP4 W4A16 linear layer on B200 (one JSON line on stdout).
+
+One step = one pass of every kernel of the hot path over the 27B-class layer
+(hidden 5120, MLP 17408), inputs resident in HBM:
+  * quantize: nvfp4_amax + nvfp4_quantize of a BF16 [17408, 5120] N(0, 0.02) tensor
+  * gemv:     batch-1 decode GEMV, NVFP4 W [17408, 5120] (headline: HBM GB/s)
+  * gemm_m32: 32-user decode GEMM, X [32, 5120]
+  * gemm_m512: 512-token prefill GEMM, X [512, 5120]
+Each kernel row is a CUDA graph of several launches over rotating weight copies
+(more bytes than the 126 MB L2 between two reads of one copy), timed with CUDA
+events on the launching stream.  `value` is the decode GEMV's algorithmic HBM
+throughput (weight nibbles + scales + x + y + g per launch / launch time), summed
+over ranks; every other kernel is reported under "kernels".
+
+--impl reference times the CPU oracle (test infrastructure) on the same
+workload: a bounded sample of decode-GEMV rows per step on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+HIDDEN, MLP = 5120, 17408
+METRIC = "NVFP4 W4A16 GEMV HBM GB/s (frac of peak); GEMM TFLOP/s at M=32/512"
+WORKLOAD = "decode GEMV NVFP4 W [N=17408, K=5120] x BF16 [1, 5120] (27B-class MLP layer)"
+
+
+def gemv_bytes(N: int, K: int) -> int:
+    """Algorithmic bytes of one decode GEMV: nibbles + scales + x + y + g."""
+    return N * K // 2 + N * K // 16 + 2 * K + 2 * N + 4
+
+
+def gemm_bytes(M: int, N: int, K: int) -> int:
+    return N * K // 2 + N * K // 16 + 2 * M * K + 2 * M * N + 4
+
+
+def quantize_bytes(N: int, K: int) -> int:
+    """amax pass (read W) + quantize pass (read W, write q and s)."""
+    return 2 * (2 * N * K) + N * K // 2 + N * K // 16
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(kernel: str, src_files):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it was
+    taken on the current source of that kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash(src_files):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ clock sampler
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        load = [v for v in sm if mx and v >= 0.0]
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------- GPU arm
+
+class _Skip(Exception):
+    pass
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    import gemm_decode_nvfp4_b200 as nv
+    import workloads
+
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    N, K = MLP, HIDDEN
+    copies = args.copies
+
+    # ---- inputs (seeded, synthetic), quantized on the GPU by the library itself
+    w_layer = workloads.weight_bf16(workloads.CONFIGS["decode"]).to(dev)
+    amax_buf = torch.zeros((1,), dtype=torch.float32, device=dev)
+    q0, s0, g0 = nv.quantize_new(w_layer)
+    del w_layer
+    qs = [q0] + [q0.clone() for _ in range(copies - 1)]
+    ss = [s0] + [s0.clone() for _ in range(copies - 1)]
+    x1 = workloads.activations(1, K, 1).to(dev).reshape(-1)
+    y1 = [torch.empty((N,), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+    X32 = workloads.activations(32, K, 3).to(dev)
+    Y32 = [torch.empty((32, N), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+    X512 = workloads.activations(512, K, 4).to(dev)
+    Y512 = torch.empty((512, N), dtype=torch.bfloat16, device=dev)
+    wq_in = workloads.to_bf16(workloads.plain_weight_f32(N, K, 4)).to(dev)
+    qq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sq = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
+    gq = torch.empty((1,), dtype=torch.float32, device=dev)
+
+    gemm_ok = args.only != "gemv"
+    gemm_err = "not run (--only gemv)"
+    try:
+        if not gemm_ok:
+            raise _Skip()
+        nv.gemm(X32, qs[0], ss[0], g0, Y32[0])
+        nv.gemm(X512, qs[0], ss[0], g0, Y512)
+        torch.cuda.synchronize()
+    except _Skip:
+        pass
+    except nv.Nvfp4Error as e:
+        gemm_ok = False
+        gemm_err = str(e)
+
+    rows = []  # (name, fn launching one graph's worth of work, launches per graph, kernels per launch)
+
+    def gemv_all():
+        for i in range(copies):
+            nv.gemv(x1, qs[i], ss[i], g0, y1[i])
+
+    def quant_all():
+        amax_buf.zero_()
+        nv.amax(wq_in, amax_buf)
+        nv.quantize(wq_in, qq, sq, gq, amax=amax_buf)
+
+    rows.append(("gemv", gemv_all, copies, 1))
+    rows.append(("quantize", quant_all, 1, 2))
+    if gemm_ok and args.only != "gemv":
+        def m32_all():
+            for i in range(copies):
+                nv.gemm(X32, qs[i], ss[i], g0, Y32[i])
+
+        def m512_all():
+            for i in range(copies):
+                nv.gemm(X512, qs[i], ss[i], g0, Y512)
+
+        rows.append(("gemm_m32", m32_all, copies, 1))
+        rows.append(("gemm_m512", m512_all, copies, 1))
+
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for name, fn, _, _ in rows:  # eager warm-up (also compiles nothing: all AOT)
+            fn()
+    stream.synchronize()
+    for name, fn, _, _ in rows:
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=stream):
+            fn()
+        graphs[name] = gph
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for name, *_ in rows:
+                graphs[name].replay()
+    stream.synchronize()
+
+    evs = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)] for name, *_ in rows}
+    step_start = torch.cuda.Event(enable_timing=True)
+    step_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clocks:
+        with torch.cuda.stream(stream):
+            step_start.record(stream)
+            for it in range(args.steps):
+                for name, *_ in rows:
+                    a, b = evs[name][it]
+                    a.record(stream)
+                    graphs[name].replay()
+                    b.record(stream)
+            step_end.record(stream)
+        stream.synchronize()
+        barrier()
+    clk = clocks.summary()
+
+    total_ms = step_start.elapsed_time(step_end)
+    per_launch_ms = {}
+    for name, _, launches, _ in rows:
+        t = sum(a.elapsed_time(b) for a, b in evs[name])
+        per_launch_ms[name] = t / (args.steps * launches)
+
+    if world > 1:
+        t = torch.tensor([total_ms] + [per_launch_ms[n] for n, *_ in rows], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t[0])
+        for i, (n, *_) in enumerate(rows):
+            per_launch_ms[n] = float(t[i + 1])
+
+    hbm = peaks["hbm_gbs"]
+    bf16_burst = peaks["bf16_tflops"]
+    kernels = {}
+    gb = gemv_bytes(N, K)
+    gemv_gbs = gb / (per_launch_ms["gemv"] * 1e-3) / 1e9
+    kernels["gemv"] = {"us": per_launch_ms["gemv"] * 1e3, "GB/s": gemv_gbs, "frac_hbm": gemv_gbs / hbm,
+                       "bytes": gb, "weight_bytes_per_token": N * K // 2 + N * K // 16}
+    qb = quantize_bytes(N, K)
+    qgbs = qb / (per_launch_ms["quantize"] * 1e-3) / 1e9
+    kernels["quantize"] = {"us": per_launch_ms["quantize"] * 1e3, "GB/s": qgbs, "frac_hbm": qgbs / hbm, "bytes": qb}
+    for name, M in (("gemm_m32", 32), ("gemm_m512", 512)):
+        if name in per_launch_ms:
+            t = per_launch_ms[name] * 1e-3
+            fl = 2.0 * M * N * K
+            byt = gemm_bytes(M, N, K)
+            kernels[name] = {"us": t * 1e6, "TFLOP/s": fl / t / 1e12, "frac_bf16": fl / t / 1e12 / bf16_burst,
+                             "GB/s": byt / t / 1e9, "frac_hbm": byt / t / 1e9 / hbm,
+                             "weight_bytes_per_token": (N * K // 2 + N * K // 16) / M}
+        elif not gemm_ok:
+            kernels[name] = {"unavailable": gemm_err}
+
+    # ---- end to end through the public API with host buffers (decode GEMV):
+    # pinned x -> device, GEMV, y -> pinned host, every step.
+    x_host = workloads.activations(1, K, 1).reshape(-1).pin_memory()
+    y_host = torch.empty((N,), dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x_host, device=dev)
+    e2e_ms = []
+    with torch.cuda.stream(stream):
+        for it in range(args.warmup + args.steps):
+            for i in range(copies):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                x_dev.copy_(x_host, non_blocking=True)
+                nv.gemv(x_dev, qs[i], ss[i], g0, y1[i])
+                y_host.copy_(y1[i], non_blocking=True)
+                b.record(stream)
+                b.synchronize()
+                if it >= args.warmup:
+                    e2e_ms.append(a.elapsed_time(b))
+    e2e_t = statistics.mean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_t = float(t[0])
+
+    launches = 0
+    for name, _, n_launch, n_kern in rows:
+        launches += args.steps * n_launch * n_kern
+
+    traffic = traffic_from_profiles("gemv", ["gemm_decode_nvfp4_b200/csrc/gemv.cu",
+                                             "gemm_decode_nvfp4_b200/csrc/nvfp4_device.cuh"])
+    out = None
+    if rank == 0:
+        out = {
+            "metric": METRIC,
+            "value": gemv_gbs * world,
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "nvfp4 weights (e2m1 + e4m3 + f32), bf16 activations, f32 accumulate",
+            "data": "synthetic (seeded numpy draws; no checkpoint)",
+            "config": {"workload": WORKLOAD, "N": N, "K": K, "M": 1, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs larger than L2: {copies} rotating weight copies "
+                             f"({copies * (N * K // 2 + N * K // 16) / 1e6:.0f} MB) per graph",
+                       "step": "quantize [17408,5120] + gemv M=1 + gemm M=32 + gemm M=512"},
+            "roofline": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gemv_gbs / hbm, "traffic": traffic,
+                         "peak_source": peaks["source"], "kernel": "gemv",
+                         "algorithmic_bytes_per_launch": gb},
+            "kernels": kernels,
+            "e2e": {"value": gb / (e2e_t * 1e-3) / 1e9 * world, "unit": "GB/s",
+                    "h2d_bytes_per_step": 2 * K, "d2h_bytes_per_step": 2 * N,
+                    "what": "per step: pinned x H2D, nvfp4_gemv, y D2H (weights resident)"},
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+        print(json.dumps(out), flush=True)
+
+    for g in graphs.values():
+        del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def _oracle_gemv_sample(n_rows: int):
+    import oracle
+    import workloads
+    cfg = workloads.CONFIGS["decode"]
+    w = workloads.to_bf16(workloads.layer_weight_f32(cfg.N, cfg.K, cfg.seed)[:n_rows])
+    q, s, g = oracle.quantize(w)
+    x = workloads.activations(1, cfg.K, cfg.seed)
+    return oracle, x, q, s, g
+
+
+def cpu_baseline(n_rows: int):
+    """The oracle's decode GEMV on a sample of rows of the decode workload,
+    timed on this host's cores; bytes counted like the GPU's (per row)."""
+    oracle, x, q, s, g = _oracle_gemv_sample(n_rows)
+    oracle.linear(x, q[:8], s[:8], g)  # load + warm
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.linear(x, q, s, g)
+        reps += 1
+        if time.perf_counter() - t0 > 2.0:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    byt = gemv_bytes(n_rows, HIDDEN)
+    return {"value": byt / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"decode GEMV rows 0..{n_rows - 1} of [17408, 5120] (fp64 oracle, {reps} reps)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    oracle, x, q, s, g = _oracle_gemv_sample(args.cpu_rows)
+    for _ in range(args.warmup):
+        oracle.linear(x, q, s, g)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.linear(x, q, s, g)
+        ts.append(time.perf_counter() - t0)
+    dt = sum(ts) / len(ts)
+    byt = gemv_bytes(args.cpu_rows, HIDDEN)
+    v = byt / dt / 1e9
+    out = {
+        "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic (seeded numpy draws)",
+        "config": {"workload": WORKLOAD, "N": MLP, "K": HIDDEN, "M": 1, "sample_rows": args.cpu_rows},
+        "impl": "reference",
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"decode GEMV rows 0..{args.cpu_rows - 1} of [17408, 5120] per step"},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out), flush=True)
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--copies", type=int, default=8, help="rotating weight copies per graph (L2 defeat)")
+    ap.add_argument("--cpu-rows", type=int, default=17408)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "gemv"],
+                    help="gemv: time only the decode GEMV and quantizer rows (profiling runs)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

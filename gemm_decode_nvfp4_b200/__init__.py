@@ -1,0 +1,185 @@
+"""Python binding of libnvfp4 (include/nvfp4.h): the NVFP4 W4A16 linear layer on B200.
+
+Argument marshalling only: every entry point takes torch CUDA tensors, checks
+dtypes and shapes, and passes raw device pointers, leading dimensions and the
+current CUDA stream to the C ABI.  All arithmetic runs in the library's CUDA
+kernels; there is no CPU path.  Importing fails loudly if the library has not
+been built (``python -m gemm_decode_nvfp4_b200.build``).
+
+Layouts follow the NVFP4 format of the pages (imp docs/quantization.md, format
+table: packed nibbles, E4M3 micro-scales per 16, FP32 tensor scale):
+q uint8 [N, K/2] (low nibble = even k), s uint8 [N, K/16], g float32 [1].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = [
+    "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
+    "gemm_workspace_size", "quantize_new", "linear", "declared_symbols",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gemm_decode_nvfp4_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_p, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+lib.nvfp4_version.argtypes, lib.nvfp4_version.restype = [], ctypes.c_int
+lib.nvfp4_last_error.argtypes, lib.nvfp4_last_error.restype = [], ctypes.c_char_p
+lib.nvfp4_status_string.argtypes, lib.nvfp4_status_string.restype = [ctypes.c_int], ctypes.c_char_p
+lib.nvfp4_amax.argtypes = [_p, _i64, _i64, _i64, _p, _p]
+lib.nvfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p]
+lib.nvfp4_gemv.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _p]
+lib.nvfp4_gemm.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]
+lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
+lib.nvfp4_gemm_workspace_size.restype = _sz
+for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm):
+    _f.restype = ctypes.c_int
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = lib.nvfp4_status_string(status).decode()
+        msg = lib.nvfp4_last_error().decode()
+        super().__init__(f"{fn}: {name}: {msg}")
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise Nvfp4Error(fn, status)
+
+
+def version() -> int:
+    return lib.nvfp4_version()
+
+
+def declared_symbols() -> list[str]:
+    """Names of the entry points include/nvfp4.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, what: str, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{what} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{what} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if t.dim() >= 1 and t.numel() > 0 and t.stride(-1) != 1:
+        raise ValueError(f"{what} must be contiguous in its last dimension")
+
+
+def _rows_ld(t: torch.Tensor):
+    return (t.shape[0], t.stride(0)) if t.dim() == 2 else (1, t.shape[-1])
+
+
+def amax(w: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """out = max(out, max|w|) for a BF16 matrix w (out: float32 [1] on the device)."""
+    _need(w, torch.bfloat16, "w")
+    _need(out, torch.float32, "out")
+    w2 = w if w.dim() == 2 else w.reshape(1, -1)
+    _check("nvfp4_amax", lib.nvfp4_amax(_ptr(w2), w2.shape[0], w2.shape[1], w2.stride(0),
+                                        _ptr(out), _stream(stream)))
+
+
+def quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch.Tensor | None,
+             amax: torch.Tensor | None = None, stream=None) -> None:
+    """RTN NVFP4 of BF16 w [N, K] into q [N, K/2] u8 and s [N, K/16] u8; g_out gets
+    g = amax / 2688.  With amax=None the tensor's own amax is used."""
+    _need(w, torch.bfloat16, "w", 2)
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    N, K = w.shape
+    if q.shape != (N, K // 2) or s.shape != (N, K // 16) or not q.is_contiguous() or not s.is_contiguous():
+        raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
+    if g_out is not None:
+        _need(g_out, torch.float32, "g_out")
+    if amax is not None:
+        _need(amax, torch.float32, "amax")
+    _check("nvfp4_quantize", lib.nvfp4_quantize(_ptr(w), N, K, w.stride(0), _ptr(amax), _ptr(q), _ptr(s),
+                                                _ptr(g_out), _stream(stream)))
+
+
+def gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, y: torch.Tensor,
+         stream=None) -> None:
+    """y[N] = bf16(g * W_deq . x) for BF16 x [K] (or [1, K])."""
+    _need(x, torch.bfloat16, "x")
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    _need(g, torch.float32, "g")
+    _need(y, torch.bfloat16, "y")
+    N, K = q.shape[0], q.shape[1] * 2
+    if x.numel() != K or y.numel() != N or not x.is_contiguous() or not y.is_contiguous():
+        raise ValueError("x must hold K and y N contiguous elements")
+    if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
+        raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
+    _check("nvfp4_gemv", lib.nvfp4_gemv(_ptr(x), _ptr(q), _ptr(s), _ptr(g), _ptr(y), N, K, _stream(stream)))
+
+
+def gemm_workspace_size(M: int, N: int, K: int) -> int:
+    return lib.nvfp4_gemm_workspace_size(M, N, K)
+
+
+def gemm(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, Y: torch.Tensor,
+         workspace: torch.Tensor | None = None, stream=None) -> None:
+    """Y [M, N] = bf16(g * X . W_deq^T) for BF16 X [M, K]."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    _need(g, torch.float32, "g")
+    _need(Y, torch.bfloat16, "Y", 2)
+    M, K = X.shape
+    N = q.shape[0]
+    if q.shape[1] * 2 != K or Y.shape != (M, N):
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
+    if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
+        raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
+    ws_bytes = 0
+    if workspace is not None:
+        _need(workspace, torch.uint8, "workspace")
+        ws_bytes = workspace.numel()
+    _check("nvfp4_gemm", lib.nvfp4_gemm(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0),
+                                        M, N, K, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+# ------------------------------------------------------ allocating helpers
+
+def quantize_new(w: torch.Tensor, amax: torch.Tensor | None = None, stream=None):
+    """Allocate q, s, g on w's device and quantize into them."""
+    N, K = w.shape
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    s = torch.empty((N, K // 16), dtype=torch.uint8, device=w.device)
+    g = torch.empty((1,), dtype=torch.float32, device=w.device)
+    quantize(w, q, s, g, amax=amax, stream=stream)
+    return q, s, g
+
+
+def linear(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, stream=None) -> torch.Tensor:
+    """Allocate Y and run the GEMM (the GEMV when X has one row)."""
+    X2 = X if X.dim() == 2 else X.reshape(1, -1)
+    Y = torch.empty((X2.shape[0], q.shape[0]), dtype=torch.bfloat16, device=X.device)
+    n_ws = gemm_workspace_size(X2.shape[0], q.shape[0], X2.shape[1])
+    ws = torch.empty((n_ws,), dtype=torch.uint8, device=X.device) if n_ws else None
+    gemm(X2, q, s, g, Y, workspace=ws, stream=stream)
+    return Y if X.dim() == 2 else Y.reshape(-1)

@@ -1,0 +1,188 @@
+// abi.cu -- the extern "C" entry points of include/nvfp4.h: host-side argument
+// validation, device capability check and dispatch to the kernels.  Nothing
+// here allocates device memory or synchronizes.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "nvfp4.h"
+#include "nvfp4_kernels.h"
+
+namespace {
+
+thread_local char t_last_error[512] = "";
+
+nvfp4_status fail(nvfp4_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+nvfp4_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(NVFP4_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return na && nb && pa < pb + nb && pb < pa + na;
+}
+
+constexpr int kMaxDevices = 64;
+int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
+int g_dev_sms[kMaxDevices];
+
+// The current device must be a B200-class part (compute capability 10.0).
+nvfp4_status check_device(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(NVFP4_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  if (g_dev_state[dev] == 0) {
+    int major = 0, minor = 0, n = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    g_dev_sms[dev] = n;
+    g_dev_state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    if (g_dev_state[dev] == 2)
+      return fail(NVFP4_ERR_UNSUPPORTED, "device %d has compute capability %d.%d; this library is built for sm_100a",
+                  dev, major, minor);
+  }
+  if (g_dev_state[dev] == 2) return fail(NVFP4_ERR_UNSUPPORTED, "device %d is not sm_100", dev);
+  *sms = g_dev_sms[dev];
+  return NVFP4_OK;
+}
+
+nvfp4_status check_k(int64_t K) {
+  if (K <= 0 || K % 16 != 0) return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 16", (long long)K);
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_version(void) { return 100; }
+
+const char* nvfp4_last_error(void) { return t_last_error; }
+
+const char* nvfp4_status_string(nvfp4_status st) {
+  switch (st) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+    case NVFP4_ERR_SHAPE: return "NVFP4_ERR_SHAPE";
+    case NVFP4_ERR_ALIGNMENT: return "NVFP4_ERR_ALIGNMENT";
+    case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE";
+  }
+  return "NVFP4_ERR_UNKNOWN";
+}
+
+nvfp4_status nvfp4_amax(const uint16_t* w, int64_t rows, int64_t cols, int64_t ldw,
+                        float* amax_inout, nvfp4_stream_t stream) {
+  if (rows < 0 || cols < 0) return fail(NVFP4_ERR_SHAPE, "negative size rows=%lld cols=%lld", (long long)rows, (long long)cols);
+  if (cols % 8 != 0) return fail(NVFP4_ERR_SHAPE, "cols=%lld must be a multiple of 8", (long long)cols);
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!w || !amax_inout) return fail(NVFP4_ERR_INVALID_ARG, "null pointer (w=%p amax=%p)", (const void*)w, (void*)amax_inout);
+  if (ldw < cols) return fail(NVFP4_ERR_INVALID_ARG, "ldw=%lld < cols=%lld", (long long)ldw, (long long)cols);
+  if (!aligned16(w) || ldw % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "w must be 16-byte aligned and ldw a multiple of 8");
+  if (!aligned4(amax_inout)) return fail(NVFP4_ERR_ALIGNMENT, "amax must be 4-byte aligned");
+  int sms = 0;
+  nvfp4_status st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_amax(w, rows, cols, ldw, amax_inout, (cudaStream_t)stream, sms);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "amax launch");
+}
+
+nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                            const float* amax, uint8_t* q, uint8_t* s, float* g_out,
+                            nvfp4_stream_t stream) {
+  nvfp4_status st = check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
+  if (!amax && !g_out) return fail(NVFP4_ERR_INVALID_ARG, "amax and g_out are both NULL");
+  if (amax && g_out && (const void*)amax == (const void*)g_out)
+    return fail(NVFP4_ERR_INVALID_ARG, "amax must not alias g_out");
+  if (N > 0 && (!w || !q || !s)) return fail(NVFP4_ERR_INVALID_ARG, "null tensor pointer");
+  if (N > 0 && ldw < K) return fail(NVFP4_ERR_INVALID_ARG, "ldw=%lld < K=%lld", (long long)ldw, (long long)K);
+  if (N > 0 && (!aligned16(w) || !aligned16(q) || !aligned16(s) || ldw % 8 != 0))
+    return fail(NVFP4_ERR_ALIGNMENT, "w, q, s must be 16-byte aligned and ldw a multiple of 8");
+  if ((amax && !aligned4(amax)) || (g_out && !aligned4(g_out)))
+    return fail(NVFP4_ERR_ALIGNMENT, "amax and g_out must be 4-byte aligned");
+  if (N > 0) {
+    const size_t wb = (size_t)((N - 1) * ldw + K) * 2, qb = (size_t)(N * K / 2), sb = (size_t)(N * K / 16);
+    if (overlaps(w, wb, q, qb) || overlaps(w, wb, s, sb) || overlaps(q, qb, s, sb) ||
+        (g_out && (overlaps(g_out, 4, q, qb) || overlaps(g_out, 4, s, sb) || overlaps(g_out, 4, w, wb))))
+      return fail(NVFP4_ERR_INVALID_ARG, "w, q, s and g_out must not overlap");
+  }
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e;
+  if (amax) {
+    e = nvfp4::launch_quantize(w, N, K, ldw, amax, q, s, g_out, cs, sms);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "quantize launch");
+  }
+  // g_out first accumulates this tensor's amax, then is overwritten with g.
+  if ((e = cudaMemsetAsync(g_out, 0, sizeof(float), cs)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  if (N > 0 && (e = nvfp4::launch_amax(w, N, K, ldw, g_out, cs, sms)) != cudaSuccess) return cuda_fail(e, "amax launch");
+  if ((e = nvfp4::launch_quantize(w, N, K, ldw, g_out, q, s, nullptr, cs, sms)) != cudaSuccess)
+    return cuda_fail(e, "quantize launch");
+  if ((e = nvfp4::launch_finalize_scale(g_out, cs)) != cudaSuccess) return cuda_fail(e, "finalize launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
+                        uint16_t* y, int64_t N, int64_t K, nvfp4_stream_t stream) {
+  nvfp4_status st = check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
+  if (K > nvfp4::kGemvMaxK) return fail(NVFP4_ERR_SHAPE, "K=%lld exceeds the GEMV limit %lld", (long long)K, (long long)nvfp4::kGemvMaxK);
+  if (N > (int64_t)0x3FFFFFFF) return fail(NVFP4_ERR_SHAPE, "N=%lld too large", (long long)N);
+  if (N == 0) return NVFP4_OK;
+  if (!x || !q || !s || !g || !y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(q) || !aligned16(s) || !aligned16(y))
+    return fail(NVFP4_ERR_ALIGNMENT, "x, q, s, y must be 16-byte aligned");
+  if (!aligned4(g)) return fail(NVFP4_ERR_ALIGNMENT, "g must be 4-byte aligned");
+  const size_t yb = (size_t)N * 2;
+  if (overlaps(y, yb, x, (size_t)K * 2) || overlaps(y, yb, q, (size_t)(N * K / 2)) ||
+      overlaps(y, yb, s, (size_t)(N * K / 16)) || overlaps(y, yb, g, 4))
+    return fail(NVFP4_ERR_INVALID_ARG, "y must not overlap x, q, s or g");
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_gemv(x, q, s, g, y, N, K, (cudaStream_t)stream);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "gemv launch");
+}
+
+size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  (void)M; (void)N; (void)K;
+  return 0;
+}
+
+nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                        const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  (void)workspace; (void)workspace_bytes;
+  nvfp4_status st = check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (M < 0 || N < 0) return fail(NVFP4_ERR_SHAPE, "negative size M=%lld N=%lld", (long long)M, (long long)N);
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!X || !q || !s || !g || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (ldx < K || ldy < N) return fail(NVFP4_ERR_INVALID_ARG, "ldx=%lld < K or ldy=%lld < N", (long long)ldx, (long long)ldy);
+  if (!aligned16(X) || !aligned16(q) || !aligned16(s) || !aligned16(Y) || ldx % 8 || ldy % 8)
+    return fail(NVFP4_ERR_ALIGNMENT, "X, q, s, Y must be 16-byte aligned and ldx, ldy multiples of 8");
+  if (!aligned4(g)) return fail(NVFP4_ERR_ALIGNMENT, "g must be 4-byte aligned");
+  if (M == 1) return nvfp4_gemv(X, q, s, g, Y, N, K, stream);
+  return fail(NVFP4_ERR_UNSUPPORTED, "M >= 2 tensor-core path not built yet");
+}
+
+}  // extern "C"

@@ -1,0 +1,24 @@
+// nvfp4_kernels.h -- internal launchers behind the C ABI (include/nvfp4.h).
+// Each returns the CUDA error of its launch; arguments are validated by the
+// caller in abi.cu before any of these runs.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+cudaError_t launch_amax(const uint16_t* w, int64_t rows, int64_t cols, int64_t ldw, float* amax,
+                        cudaStream_t stream, int sms);
+cudaError_t launch_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                            const float* amax, uint8_t* q, uint8_t* s, float* g_out,
+                            cudaStream_t stream, int sms);
+cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream);
+cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
+                        uint16_t* y, int64_t N, int64_t K, cudaStream_t stream);
+
+// Largest K the GEMV accepts (x is staged in shared memory as fp32).
+constexpr int64_t kGemvMaxK = 49152;
+
+}  // namespace nvfp4

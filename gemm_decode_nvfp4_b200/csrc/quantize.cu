@@ -1,0 +1,150 @@
+// quantize.cu -- tensor amax and round-to-nearest BF16 -> NVFP4 quantization.
+//
+// Follows imp docs/quantization.md, "imp-quantize" section (plain
+// round-to-nearest from the absmax of each 16-block, E4M3 micro-scale, FP32
+// tensor scale) and the model card "Qwen3.8-27B-NVFP4", paragraph after
+// "What is quantized" (merged layers share the tensor scale: the caller
+// accumulates one amax over all members).
+//
+// Both kernels stream HBM once: amax reads W (2 B/element); quantize reads W
+// and writes 0.5 + 1/16 B/element.  Each thread owns whole 16-element blocks
+// (32 B in, 8 B of codes + 1 scale byte out), so loads are 16-byte vectors
+// that are contiguous across a warp and blocks never straddle threads.
+#include "nvfp4_kernels.h"
+#include "nvfp4_device.cuh"
+
+namespace nvfp4 {
+
+namespace {
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float absmax8(uint4 v, float m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, fabsf(bf16lo_to_float(w[i])));
+    m = fmaxf(m, fabsf(bf16hi_to_float(w[i])));
+  }
+  return m;
+}
+
+// amax over rows x cols (cols % 8 == 0), atomically max-merged into *out.
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ w, int64_t rows,
+                                                   int64_t cols, int64_t ldw,
+                                                   float* __restrict__ out) {
+  __shared__ float red[8];
+  const int64_t vpr = cols / 8;
+  const int64_t total = rows * vpr;
+  float m = 0.0f;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = t / vpr, c = (t - r * vpr) * 8;
+    m = absmax8(ld_stream_v4(w + r * ldw + c), m);
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+    m = warp_max(m);
+    // non-negative floats order like their bit patterns
+    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(m));
+  }
+}
+
+// One 16-element block: scale byte and 8 code bytes.
+__device__ __forceinline__ void quantize_block(const float (&f)[16], float g, uint32_t& scale,
+                                               uint2& codes) {
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(f[i]));
+  uint32_t sc = 0;
+  if (g != 0.0f) sc = float_to_e4m3_satfinite(__fdiv_rn(__fdiv_rn(amax_b, 6.0f), g));
+  const float d = __fmul_rn(e4m3_to_float(sc), g);
+  uint32_t c[8];
+  if (d == 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = 0;
+  } else {
+    const float r = __frcp_rn(d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // +-0 keeps its sign even when r overflowed to infinity
+      const float lo = (f[2 * i] == 0.0f) ? f[2 * i] : __fmul_rn(f[2 * i], r);
+      const float hi = (f[2 * i + 1] == 0.0f) ? f[2 * i + 1] : __fmul_rn(f[2 * i + 1], r);
+      c[i] = float2_to_e2m1x2_satfinite(lo, hi);
+    }
+  }
+  scale = sc;
+  codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+  codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+}
+
+__global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ w, int64_t N,
+                                                       int64_t K, int64_t ldw,
+                                                       const float* __restrict__ amax,
+                                                       uint8_t* __restrict__ q,
+                                                       uint8_t* __restrict__ s,
+                                                       float* __restrict__ g_out) {
+  const float g = __fdiv_rn(*amax, 2688.0f);
+  if (g_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  const int64_t bpr = K / 16;
+  const int64_t total = N * bpr;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = t / bpr, b = t - n * bpr;
+    const uint16_t* src = w + n * ldw + b * 16;
+    const uint4 v0 = ld_stream_v4(src), v1 = ld_stream_v4(src + 8);
+    const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = bf16lo_to_float(wv[i]);
+      f[2 * i + 1] = bf16hi_to_float(wv[i]);
+    }
+    uint32_t sc;
+    uint2 codes;
+    quantize_block(f, g, sc, codes);
+    *reinterpret_cast<uint2*>(q + n * (K / 2) + b * 8) = codes;
+    s[n * bpr + b] = static_cast<uint8_t>(sc);
+  }
+}
+
+__global__ void finalize_scale_kernel(float* amax_then_g) {
+  *amax_then_g = __fdiv_rn(*amax_then_g, 2688.0f);
+}
+
+int grid_for(int64_t work_items, int sms) {
+  const int64_t blocks = (work_items + 255) / 256;
+  const int64_t cap = (int64_t)sms * 8;
+  return (int)(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
+}
+
+}  // namespace
+
+cudaError_t launch_amax(const uint16_t* w, int64_t rows, int64_t cols, int64_t ldw, float* amax,
+                        cudaStream_t stream, int sms) {
+  const int grid = grid_for(rows * (cols / 8), sms);
+  amax_kernel<<<grid, 256, 0, stream>>>(w, rows, cols, ldw, amax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                            const float* amax, uint8_t* q, uint8_t* s, float* g_out,
+                            cudaStream_t stream, int sms) {
+  const int grid = grid_for(N * (K / 16), sms);
+  quantize_kernel<<<grid, 256, 0, stream>>>(w, N, K, ldw, amax, q, s, g_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream) {
+  finalize_scale_kernel<<<1, 1, 0, stream>>>(amax_then_g);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,155 @@
+/*
+ * nvfp4.h -- C ABI of the NVFP4 weight-only (W4A16) linear-layer library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (web pages, by title and section):
+ *   - "Raphael Friedmann" home page, NVFP4 bit-level graphic: a weight is an
+ *     E2M1 nibble (1 sign, 2 exponent, 1 mantissa bit), every 16 values share
+ *     an FP8 scale and the tensor has one FP32 scale.
+ *   - imp docs/quantization.md, format table and "imp-quantize" section: the
+ *     packed layout (.weight U8 nibbles, .weight_scale F8_E4M3 per 16,
+ *     .weight_scale_2 F32) and plain round-to-nearest from the block absmax;
+ *     "Dense layers" pipeline: decode GEMV and prefill GEMM read it directly.
+ *   - model card "Qwen3.8-27B-NVFP4 (compressed-tensors)", "What is quantized"
+ *     and the paragraph after it: weight-only (activations stay BF16), group
+ *     size 16, merged q/k/v and gate/up layers share one tensor scale.
+ *
+ * Layouts (all row-major, no padding inside a row):
+ *   W  BF16 [N, K]  with leading dimension ldw (elements)       (quantizer input)
+ *   q  u8   [N, K/2] byte j of row n holds element 2j in its low nibble and
+ *                    element 2j+1 in its high nibble (E2M1 codes)
+ *   s  u8   [N, K/16] E4M3 scale of elements 16j .. 16j+15 of row n
+ *   g  fp32 scalar   dequantization multiplier, g = amax / (6 * 448)
+ *   X  BF16 [M, K] with leading dimension ldx;  Y BF16 [M, N] with ldy
+ *   Y[m, n] = bf16_rn( g * sum_j e4m3(s[n, j]) * sum_i e2m1(q[n, 16j+i]) * X[m, 16j+i] )
+ *   accumulated in fp32.
+ *
+ * Conventions of every entry point:
+ *   - Pointers to tensors are DEVICE pointers owned by the caller; the library
+ *     keeps no pointer after the call returns and allocates no device memory.
+ *     BF16 tensors are passed as uint16_t bit patterns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; the call does not synchronize.
+ *   - Arguments are validated on the host before anything is launched.  On
+ *     failure nothing is enqueued, a status other than NVFP4_OK is returned and
+ *     nvfp4_last_error() describes it.  No call aborts or throws.
+ *   - Tensor pointers must be 16-byte aligned and scalar pointers (g, amax)
+ *     4-byte aligned; leading dimensions are multiples of 8 elements.  K is a
+ *     positive multiple of 16 (one scale per 16).
+ *   - Calls on the same stream are ordered; calls on different streams that
+ *     write the same buffers race.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, kept opaque so that this header needs no CUDA headers. */
+typedef void* nvfp4_stream_t;
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* null pointer, negative size, aliasing outputs */
+  NVFP4_ERR_SHAPE = 2,       /* K not a positive multiple of 16, M/N < 0, size too large */
+  NVFP4_ERR_ALIGNMENT = 3,   /* pointer not 16-byte aligned, leading dim not a multiple of 8 */
+  NVFP4_ERR_UNSUPPORTED = 4, /* current device is not compute capability 10.0 (B200) */
+  NVFP4_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  NVFP4_ERR_WORKSPACE = 6    /* workspace missing or smaller than nvfp4_gemm_workspace_size() */
+} nvfp4_status;
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+NVFP4_API int nvfp4_version(void);
+
+/* Message of the most recent failed call made by this host thread ("" if none).
+ * The string is owned by the library and stays valid until the thread's next
+ * failing call. */
+NVFP4_API const char* nvfp4_last_error(void);
+
+/* Short name of a status code. */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status status);
+
+/*
+ * Tensor amax: *amax_inout = max(*amax_inout, max |W|) over a BF16 [rows, cols]
+ * matrix (leading dimension ldw).  Follows the FP32 per-tensor scale of the
+ * NVFP4 graphic on the "Raphael Friedmann" home page and the shared-scale rule
+ * of the model card "Qwen3.8-27B-NVFP4" (merged members share one amax): zero
+ * *amax_inout once, then call this once per member to get the merged amax.
+ * amax_inout is one device fp32; the update is an atomic max, so concurrent
+ * calls on one accumulator are safe.  cols must be a multiple of 8.
+ * rows == 0 or cols == 0 is a no-op.
+ */
+NVFP4_API nvfp4_status nvfp4_amax(const uint16_t* w, int64_t rows, int64_t cols, int64_t ldw,
+                        float* amax_inout, nvfp4_stream_t stream);
+
+/*
+ * Round-to-nearest NVFP4 quantization (imp docs/quantization.md, "imp-quantize":
+ * plain round-to-nearest from the block absmax, no calibration) of a BF16
+ * W [N, K] (leading dimension ldw) into q [N, K/2] and s [N, K/16].
+ *
+ * Arithmetic (IEEE fp32, round to nearest even, no contraction), per 16-block b
+ * of row n with amax_b = max |w| over the block:
+ *   g   = amax / 2688                      (written to *g_out)
+ *   s   = E4M3_rne_satfinite((amax_b / 6) / g),   s = 0 when g == 0
+ *   d   = e4m3(s) * g;   all 16 codes 0x0 when d == 0, else with r = 1 / d:
+ *   code = E2M1_rne_satfinite(w * r)  (ties to the even code, sign kept,
+ *          |w * r| > 6 saturates to 6; w == +-0 gives 0x0 / 0x8)
+ *
+ * amax: device fp32 holding the tensor amax to use (for a merged layer, the max
+ *   over all members, as accumulated by nvfp4_amax).  NULL = compute this
+ *   tensor's own amax first (then g_out is used as the accumulator and is
+ *   overwritten with g at the end).  amax must not alias g_out.
+ * g_out: device fp32 receiving g.  May be NULL when amax is given.
+ * Output bytes are bit-exact functions of the inputs (deterministic).
+ * N == 0 is a no-op apart from writing *g_out.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                            const float* amax, uint8_t* q, uint8_t* s, float* g_out,
+                            nvfp4_stream_t stream);
+
+/*
+ * Batch-1 decode GEMV, y[n] = bf16_rn(g * sum_k W_deq[n, k] * x[k]) with fp32
+ * accumulation ("Dense layers" pipeline of imp docs/quantization.md: the decode
+ * path reads packed FP4 directly; weight-only per the model card).
+ * x: BF16 [K]; q, s as above; g: device fp32; y: BF16 [N].
+ * y must not overlap x, q or s.  N == 0 is a no-op.
+ * Limits: K <= 49152 (x is staged in shared memory).
+ */
+NVFP4_API nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s,
+                        const float* g, uint16_t* y, int64_t N, int64_t K,
+                        nvfp4_stream_t stream);
+
+/*
+ * GEMM Y = X . W^T for M >= 1 rows of activations (32-user batched decode and
+ * 512-token prefill of the model card "Qwen3.8-27B-NVFP4", "Measurements"),
+ * same arithmetic as nvfp4_gemv per output.  M == 1 runs the GEMV.  M >= 2 runs
+ * on the tensor cores (tcgen05, BF16 operands, fp32 accumulation in tensor
+ * memory); the dequantized weights e2m1 * e4m3 are exact in BF16, g is applied
+ * in fp32 in the epilogue.
+ * workspace: device scratch of nvfp4_gemm_workspace_size(M, N, K) bytes, may be
+ *   NULL when that size is 0.
+ * Y must not overlap X, q or s.  M == 0 or N == 0 is a no-op.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                        const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                        int64_t K, void* workspace, size_t workspace_bytes,
+                        nvfp4_stream_t stream);
+
+/* Bytes of workspace nvfp4_gemm needs for this shape (0 if none). */
+NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

@@ -1,0 +1,71 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/nvfp4.h declares, and rejects bad arguments before touching a GPU.
+No call here reaches a kernel launch (all fail validation first)."""
+import ctypes
+
+import pytest
+
+import gemm_decode_nvfp4_b200 as nv
+
+OK, INVALID, SHAPE, ALIGN = 0, 1, 2, 3
+A = 1 << 20  # a fake, 16-byte aligned "device address": never dereferenced here
+
+
+def test_exports_every_declared_symbol():
+    names = nv.declared_symbols()
+    assert set(names) >= {"nvfp4_amax", "nvfp4_quantize", "nvfp4_gemv", "nvfp4_gemm",
+                          "nvfp4_gemm_workspace_size", "nvfp4_last_error", "nvfp4_version",
+                          "nvfp4_status_string"}
+    raw = ctypes.CDLL(nv.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_version_and_status_strings():
+    assert nv.version() >= 100
+    assert nv.lib.nvfp4_status_string(0) == b"NVFP4_OK"
+    assert nv.lib.nvfp4_status_string(3) == b"NVFP4_ERR_ALIGNMENT"
+    assert nv.lib.nvfp4_status_string(99) == b"NVFP4_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("K", [0, -16, 8, 24, 100])
+def test_bad_k_rejected(K):
+    assert nv.lib.nvfp4_gemv(A, A, A, A, A + 4096, 16, K, None) == SHAPE
+    assert nv.lib.nvfp4_quantize(A, 16, K, 64, A, A, A, A + 64, None) == SHAPE
+    assert nv.lib.nvfp4_gemm(A, 64, A, A, A, A, 64, 4, 16, K, None, 0, None) == SHAPE
+    assert b"multiple of 16" in nv.lib.nvfp4_last_error()
+
+
+def test_gemv_validation():
+    assert nv.lib.nvfp4_gemv(A, A, A, A, A, -1, 64, None) == SHAPE
+    assert nv.lib.nvfp4_gemv(A, A, A, A, A, 0, 64, None) == OK          # no-op, no device needed
+    assert nv.lib.nvfp4_gemv(None, A, A, A, A, 4, 64, None) == INVALID
+    assert nv.lib.nvfp4_gemv(A + 8, A, A, A, A + 4096, 4, 64, None) == ALIGN
+    assert nv.lib.nvfp4_gemv(A, A, A, A + 2, A + 4096, 4, 64, None) == ALIGN
+    assert nv.lib.nvfp4_gemv(A, A, A, A, A + 4096, 4, 49152 + 16, None) == SHAPE
+    # y overlapping x
+    assert nv.lib.nvfp4_gemv(A, A + 8192, A + 16384, A + 32768, A + 16, 4, 64, None) == INVALID
+
+
+def test_quantize_validation():
+    assert nv.lib.nvfp4_quantize(A, 4, 64, 64, None, A + 4096, A + 8192, None, None) == INVALID
+    assert nv.lib.nvfp4_quantize(A, 4, 64, 64, A, A + 4096, A + 8192, A, None) == INVALID   # alias
+    assert nv.lib.nvfp4_quantize(A, 4, 64, 32, A + 100, A + 4096, A + 8192, None, None) == INVALID  # ldw < K
+    assert nv.lib.nvfp4_quantize(A, 4, 64, 68, A + 100, A + 4096, A + 8192, None, None) == ALIGN
+    assert nv.lib.nvfp4_quantize(A, -1, 64, 64, A + 100, A + 4096, A + 8192, None, None) == SHAPE
+    # q overlapping w
+    assert nv.lib.nvfp4_quantize(A, 4, 64, 64, A + 100000, A + 16, A + 8192, None, None) == INVALID
+
+
+def test_amax_validation():
+    assert nv.lib.nvfp4_amax(A, 4, 12, 16, A + 4096, None) == SHAPE
+    assert nv.lib.nvfp4_amax(A, 0, 16, 16, None, None) == OK
+    assert nv.lib.nvfp4_amax(None, 4, 16, 16, A, None) == INVALID
+    assert nv.lib.nvfp4_amax(A + 2, 4, 16, 16, A + 4096, None) == ALIGN
+
+
+def test_gemm_validation():
+    assert nv.lib.nvfp4_gemm(A, 64, A, A, A, A, 64, 0, 64, 64, None, 0, None) == OK
+    assert nv.lib.nvfp4_gemm(A, 32, A, A, A, A, 64, 4, 64, 64, None, 0, None) == INVALID  # ldx < K
+    assert nv.lib.nvfp4_gemm(A, 72, A, A, A, A, 68, 4, 64, 64, None, 0, None) == ALIGN   # ldy % 8
+    assert nv.lib.nvfp4_gemm(A, 64, A, A, A, None, 64, 4, 64, 64, None, 0, None) == INVALID
