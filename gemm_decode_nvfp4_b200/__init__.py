@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
-    "gemm_workspace_size", "quantize_new", "linear", "declared_symbols",
+    "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,8 @@ lib.nvfp4_gemv.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _p]
 lib.nvfp4_gemm.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]
 lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
 lib.nvfp4_gemm_workspace_size.restype = _sz
-for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm):
+lib.nvfp4_check_device_errors.argtypes = []
+for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_check_device_errors):
     _f.restype = ctypes.c_int
 
 
@@ -57,6 +58,11 @@ class Nvfp4Error(RuntimeError):
 def _check(fn: str, status: int) -> None:
     if status != 0:
         raise Nvfp4Error(fn, status)
+
+
+def check_device_errors() -> None:
+    """Raise if a tensor-core GEMM CTA gave up on a bounded pipeline wait."""
+    _check("nvfp4_check_device_errors", lib.nvfp4_check_device_errors())
 
 
 def version() -> int:

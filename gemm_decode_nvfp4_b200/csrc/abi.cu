@@ -26,6 +26,7 @@ nvfp4_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned2(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1u) == 0; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
@@ -81,6 +82,7 @@ const char* nvfp4_status_string(nvfp4_status st) {
     case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
     case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
     case NVFP4_ERR_WORKSPACE: return "NVFP4_ERR_WORKSPACE";
+    case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
   }
   return "NVFP4_ERR_UNKNOWN";
 }
@@ -149,8 +151,9 @@ nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
   if (N > (int64_t)0x3FFFFFFF) return fail(NVFP4_ERR_SHAPE, "N=%lld too large", (long long)N);
   if (N == 0) return NVFP4_OK;
   if (!x || !q || !s || !g || !y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
-  if (!aligned16(x) || !aligned16(q) || !aligned16(s) || !aligned16(y))
-    return fail(NVFP4_ERR_ALIGNMENT, "x, q, s, y must be 16-byte aligned");
+  if (!aligned16(x) || !aligned16(q) || !aligned16(s))
+    return fail(NVFP4_ERR_ALIGNMENT, "x, q, s must be 16-byte aligned");
+  if (!aligned2(y)) return fail(NVFP4_ERR_ALIGNMENT, "y must be 2-byte aligned");
   if (!aligned4(g)) return fail(NVFP4_ERR_ALIGNMENT, "g must be 4-byte aligned");
   const size_t yb = (size_t)N * 2;
   if (overlaps(y, yb, x, (size_t)K * 2) || overlaps(y, yb, q, (size_t)(N * K / 2)) ||
@@ -178,11 +181,41 @@ nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const 
   if (M == 0 || N == 0) return NVFP4_OK;
   if (!X || !q || !s || !g || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
   if (ldx < K || ldy < N) return fail(NVFP4_ERR_INVALID_ARG, "ldx=%lld < K or ldy=%lld < N", (long long)ldx, (long long)ldy);
-  if (!aligned16(X) || !aligned16(q) || !aligned16(s) || !aligned16(Y) || ldx % 8 || ldy % 8)
-    return fail(NVFP4_ERR_ALIGNMENT, "X, q, s, Y must be 16-byte aligned and ldx, ldy multiples of 8");
+  if (!aligned16(X) || !aligned16(q) || !aligned16(s) || ldx % 8)
+    return fail(NVFP4_ERR_ALIGNMENT, "X, q, s must be 16-byte aligned and ldx a multiple of 8");
+  if (!aligned2(Y)) return fail(NVFP4_ERR_ALIGNMENT, "Y must be 2-byte aligned");
   if (!aligned4(g)) return fail(NVFP4_ERR_ALIGNMENT, "g must be 4-byte aligned");
+  {
+    const size_t xb = (size_t)((M - 1) * ldx + K) * 2, yb = (size_t)((M - 1) * ldy + N) * 2;
+    if (overlaps(Y, yb, X, xb) || overlaps(Y, yb, q, (size_t)(N * K / 2)) || overlaps(Y, yb, s, (size_t)(N * K / 16)) ||
+        overlaps(Y, yb, g, 4))
+      return fail(NVFP4_ERR_INVALID_ARG, "Y must not overlap X, q, s or g");
+  }
   if (M == 1) return nvfp4_gemv(X, q, s, g, Y, N, K, stream);
-  return fail(NVFP4_ERR_UNSUPPORTED, "M >= 2 tensor-core path not built yet");
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e;
+  if (nvfp4::gemm_tc_supported(M, N, K)) {
+    e = nvfp4::launch_gemm_tc(X, ldx, q, s, g, Y, ldy, M, N, K, (cudaStream_t)stream);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "tensor-core gemm launch");
+  }
+  // K not a multiple of 256: one decode GEMV per row of X (same arithmetic).
+  if (K > nvfp4::kGemvMaxK) return fail(NVFP4_ERR_SHAPE, "K=%lld: the GEMM needs K %% 256 == 0 or K <= %lld",
+                                        (long long)K, (long long)nvfp4::kGemvMaxK);
+  for (int64_t m = 0; m < M; ++m) {
+    e = nvfp4::launch_gemv(X + m * ldx, q, s, g, Y + m * ldy, N, K, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
+  }
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_check_device_errors(void) {
+  unsigned int n = 0;
+  cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error counter");
+  if (n) return fail(NVFP4_ERR_TIMEOUT, "%u tensor-core GEMM CTA(s) gave up on a pipeline wait", n);
+  return NVFP4_OK;
 }
 
 }  // extern "C"

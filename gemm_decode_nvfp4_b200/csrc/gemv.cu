@@ -4,15 +4,24 @@
 // NVFP4 GEMV reading the packed nibbles, E4M3 micro-scales and FP32 tensor
 // scale directly) with BF16 activations (model card "Qwen3.8-27B-NVFP4",
 // "What is quantized": weight-only).  The pages' kernel targets sm_120 with a
-// prmt register LUT; here the sm_100a cvt.rn.f16x2.e2m1x2 instruction decodes
-// two codes per instruction (exactly, sign included) and the products are
-// accumulated with packed fp32x2 FMAs.
+// prmt register LUT; on sm_100a the weight decode is one
+// cvt.rn.f16x2.e2m1x2 per two codes (exact, sign included) and each product
+// is one mixed-precision fma.rn.f32.f16 (f16 x f16 -> fp32 accumulator),
+// which issues at the full FFMA rate.
+//
+// x is staged once per CTA in shared memory.  For the f16 operand it is
+// scaled by a power of two 2^e chosen from max|x| so that every element is
+// exactly representable in f16 (BF16 has 8 significant bits, f16 11): this
+// holds when all non-zero |x| lie within 2^32 of max|x| and x is finite, which
+// the CTA checks while staging.  Otherwise the CTA takes the exact fp32 path
+// (x in fp32, codes -> f16 -> fp32, packed fp32x2 FMAs).  Either way every
+// product is exact and the accumulation is fp32; the result is
+// y = bf16_rn(2^-e * (g * acc)).
 //
 // Work split: a warp owns R consecutive rows; lane l reads the 16-byte chunks
 // l, l+32, ... of each row (512 contiguous bytes per warp-load, one 16-bit
-// scale load per chunk).  x is staged once per CTA in shared memory as fp32.
-// Per chunk and row: 8 cvt + 16 f16->f32 + 16 FFMA2 for 32 weights, plus two
-// block sums and two scale FMAs.  The weight stream (0.5625 B/weight) is the
+// scale load per chunk), with the next chunk's loads in flight while the
+// current one is reduced.  The weight stream (0.5625 B/weight) is the
 // roofline: HBM bandwidth.
 #include "nvfp4_kernels.h"
 #include "nvfp4_device.cuh"
@@ -24,23 +33,42 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 
-// CB = bytes of packed codes per lane per step (16, or 8 when K % 32 != 0).
-template <int R, int CB>
-__global__ void __launch_bounds__(kThreads) gemv_kernel(const uint16_t* __restrict__ x,
-                                                        const uint8_t* __restrict__ q,
-                                                        const uint8_t* __restrict__ s,
-                                                        const float* __restrict__ g,
-                                                        uint16_t* __restrict__ y, int N, int K) {
-  extern __shared__ __align__(16) float xs[];  // K fp32
-  constexpr int kElems = 2 * CB;               // weights per lane-chunk
-  constexpr int kBlocks = kElems / 16;         // scales per lane-chunk (2 or 1)
+// c + lo(a)*lo(b) + hi(a)*hi(b) with a, b f16x2 pairs, in fp32 (products exact).
+__device__ __forceinline__ float fma2_f16_f32(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.f16 t, al, bl, %3;\n\tfma.rn.f32.f16 %0, ah, bh, t;\n\t}"
+      : "=f"(d)
+      : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+
+// floor(log2(v)) of a non-zero, finite BF16 magnitude given by its 15 low bits.
+__device__ __forceinline__ int bf16_ilogb(uint32_t a) {
+  return a >= 0x80u ? (int)(a >> 7) - 127 : (31 - __clz((int)a)) - 133;
+}
+
+// 2^k as fp32 for k in [-126, 127].
+__device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+
+template <int R, int CB, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __restrict__ x,
+                                                              const uint8_t* __restrict__ q,
+                                                              const uint8_t* __restrict__ s,
+                                                              const float* __restrict__ g,
+                                                              uint16_t* __restrict__ y, int N, int K) {
+  extern __shared__ __align__(16) uint8_t xsm[];  // K f16 (fast path) or K fp32 (exact path)
+  __shared__ uint32_t red_max[kWarps], red_min[kWarps];
+  constexpr int kBlocks = (2 * CB) / 16;  // scales per lane-chunk (2 or 1)
+  constexpr int kWords = CB / 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = (blockIdx.x * kWarps + warp) * R;
   const int row_bytes = K >> 1;
   const int row_scales = K >> 4;
   const int steps = (row_bytes + 32 * CB - 1) / (32 * CB);
 
-  auto load = [&](int step, uint32_t (&wq)[R][CB / 4], uint32_t (&ws)[R]) {
+  auto load = [&](int step, uint32_t (&wq)[R][kWords], uint32_t (&ws)[R]) {
     const int off = step * 32 * CB + lane * CB;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -59,22 +87,66 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const uint16_t* __restri
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < CB / 4; ++i) wq[r][i] = 0;
+        for (int i = 0; i < kWords; ++i) wq[r][i] = 0;
         ws[r] = 0;
       }
     }
   };
 
-  uint32_t wq[R][CB / 4], ws[R];
+  uint32_t wq[R][kWords], ws[R];
   load(0, wq, ws);  // first weights in flight before x is staged
 
+  // ---- range of |x| (bit patterns of non-negative BF16 order like values)
+  uint32_t mx = 0, mn = 0xFFFFu;
   for (int i = threadIdx.x; i < (K >> 3); i += kThreads) {
     const uint4 v = *reinterpret_cast<const uint4*>(x + 8 * i);
-    float4* dst = reinterpret_cast<float4*>(xs) + 2 * i;
-    dst[0] = make_float4(bf16lo_to_float(v.x), bf16hi_to_float(v.x), bf16lo_to_float(v.y),
-                         bf16hi_to_float(v.y));
-    dst[1] = make_float4(bf16lo_to_float(v.z), bf16hi_to_float(v.z), bf16lo_to_float(v.w),
-                         bf16hi_to_float(v.w));
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
+      mx = max(mx, max(lo, hi));
+      mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
+    }
+  }
+  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+  mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+  if (lane == 0) { red_max[warp] = mx; red_min[warp] = mn; }
+  __syncthreads();
+  mx = red_max[0]; mn = red_min[0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) { mx = max(mx, red_max[w]); mn = min(mn, red_min[w]); }
+  bool fast = true;
+  int e = 0;
+  if (mx >= 0x7F80u) {
+    fast = false;                       // inf or NaN in x
+  } else if (mx != 0) {
+    const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
+    e = 15 - hi_exp;                    // max |x| * 2^e in [2^15, 2^16)
+    fast = hi_exp - lo_exp <= 32;       // smallest non-zero |x| * 2^e >= 2^-17
+  }
+
+  // ---- stage x
+  if (fast) {
+    const int e1 = e / 2, e2 = e - e1;  // two exact power-of-two steps
+    const float m1 = exp2i(e1), m2 = exp2i(e2);
+    for (int i = threadIdx.x; i < (K >> 3); i += kThreads) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x + 8 * i);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 h = __floats2half2_rn(bf16lo_to_float(w4[j]) * m1 * m2, bf16hi_to_float(w4[j]) * m1 * m2);
+        o[j] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(xsm)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  } else {
+    for (int i = threadIdx.x; i < (K >> 3); i += kThreads) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x + 8 * i);
+      float4* dst = reinterpret_cast<float4*>(xsm) + 2 * i;
+      dst[0] = make_float4(bf16lo_to_float(v.x), bf16hi_to_float(v.x), bf16lo_to_float(v.y), bf16hi_to_float(v.y));
+      dst[1] = make_float4(bf16lo_to_float(v.z), bf16hi_to_float(v.z), bf16lo_to_float(v.w), bf16hi_to_float(v.w));
+    }
   }
   __syncthreads();
 
@@ -83,45 +155,62 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const uint16_t* __restri
   for (int r = 0; r < R; ++r) acc[r] = 0.0f;
 
   for (int step = 0; step < steps; ++step) {
-    uint32_t nq[R][CB / 4], ns[R];
+    uint32_t nq[R][kWords], ns[R];
     if (step + 1 < steps) load(step + 1, nq, ns);
     const int off = step * 32 * CB + lane * CB;
     if (off < row_bytes) {
-      const float* xp = xs + 2 * off;
-      float2 part[R][kBlocks];
+      float part[R][kBlocks];
 #pragma unroll
       for (int r = 0; r < R; ++r)
 #pragma unroll
-        for (int b = 0; b < kBlocks; ++b) part[r][b] = make_float2(0.0f, 0.0f);
+        for (int b = 0; b < kBlocks; ++b) part[r][b] = 0.0f;
+      if (fast) {
+        const uint4* xp = reinterpret_cast<const uint4*>(xsm) + (2 * off) / 8;
 #pragma unroll
-      for (int wi = 0; wi < CB / 4; ++wi) {  // 8 weights per 32-bit word
-        const float4 xa = reinterpret_cast<const float4*>(xp)[2 * wi];
-        const float4 xb = reinterpret_cast<const float4*>(xp)[2 * wi + 1];
-        const float2 x01 = make_float2(xa.x, xa.y), x23 = make_float2(xa.z, xa.w);
-        const float2 x45 = make_float2(xb.x, xb.y), x67 = make_float2(xb.z, xb.w);
-        const int b = wi / 2;  // two words per 16-block
+        for (int wi = 0; wi < kWords; ++wi) {  // 8 weights per 32-bit word
+          const uint4 xv = xp[wi];
+          const int b = wi / 2;
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const uint32_t word = wq[r][wi];
-          float2& p = part[r][b];
-          p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<0>(word)), x01, p);
-          p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<1>(word)), x23, p);
-          p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<2>(word)), x45, p);
-          p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<3>(word)), x67, p);
+          for (int r = 0; r < R; ++r) {
+            const uint32_t word = wq[r][wi];
+            float p = part[r][b];
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
+            part[r][b] = p;
+          }
+        }
+      } else {
+        const float4* xp = reinterpret_cast<const float4*>(xsm) + (2 * off) / 4;
+#pragma unroll
+        for (int wi = 0; wi < kWords; ++wi) {
+          const float4 xa = xp[2 * wi], xb = xp[2 * wi + 1];
+          const int b = wi / 2;
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const uint32_t word = wq[r][wi];
+            float2 p = make_float2(0.0f, 0.0f);
+            p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<0>(word)), make_float2(xa.x, xa.y), p);
+            p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<1>(word)), make_float2(xa.z, xa.w), p);
+            p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<2>(word)), make_float2(xb.x, xb.y), p);
+            p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<3>(word)), make_float2(xb.z, xb.w), p);
+            part[r][b] += p.x + p.y;
+          }
         }
       }
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const float2 sc = f16x2_to_float2(e4m3x2_to_f16x2(ws[r]));
-        acc[r] = fmaf(part[r][0].x + part[r][0].y, sc.x, acc[r]);
-        if constexpr (kBlocks == 2) acc[r] = fmaf(part[r][1].x + part[r][1].y, sc.y, acc[r]);
+        acc[r] = fmaf(part[r][0], sc.x, acc[r]);
+        if constexpr (kBlocks == 2) acc[r] = fmaf(part[r][1], sc.y, acc[r]);
       }
     }
     if (step + 1 < steps) {
 #pragma unroll
       for (int r = 0; r < R; ++r) {
 #pragma unroll
-        for (int i = 0; i < CB / 4; ++i) wq[r][i] = nq[r][i];
+        for (int i = 0; i < kWords; ++i) wq[r][i] = nq[r][i];
         ws[r] = ns[r];
       }
     }
@@ -142,19 +231,27 @@ __global__ void __launch_bounds__(kThreads) gemv_kernel(const uint16_t* __restri
       if (lane == r) v = acc[r];
     const int row = row0 + lane;
     if (row < N) {
-      const __nv_bfloat16 o = __float2bfloat16_rn(v * gv);
+      const float out = fast ? ldexpf(v * gv, -e) : v * gv;
+      const __nv_bfloat16 o = __float2bfloat16_rn(out);
       y[row] = *reinterpret_cast<const uint16_t*>(&o);
     }
   }
 }
 
-template <int R, int CB>
-cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
-                   uint16_t* y, int N, int K, cudaStream_t stream) {
+template <int R, int CB, int MINB>
+cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y, int N,
+                   int K, cudaStream_t stream) {
   const size_t smem = (size_t)K * sizeof(float);
-  auto kern = gemv_kernel<R, CB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = gemv_kernel<R, CB, MINB>;
+  static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || smem_set[dev] < (int)smem) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) smem_set[dev] = (int)smem;
+  }
   const int rows_per_cta = kWarps * R;
   const int grid = (N + rows_per_cta - 1) / rows_per_cta;
   kern<<<grid, kThreads, smem, stream>>>(x, q, s, g, y, N, K);
@@ -165,8 +262,8 @@ cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const 
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, cudaStream_t stream) {
-  if (K % 32 == 0) return launch<4, 16>(x, q, s, g, y, (int)N, (int)K, stream);
-  return launch<4, 8>(x, q, s, g, y, (int)N, (int)K, stream);
+  if (K % 32 == 0) return launch<4, 16, 3>(x, q, s, g, y, (int)N, (int)K, stream);
+  return launch<4, 8, 3>(x, q, s, g, y, (int)N, (int)K, stream);
 }
 
 }  // namespace nvfp4

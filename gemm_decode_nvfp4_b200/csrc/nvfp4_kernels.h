@@ -18,6 +18,13 @@ cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream);
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, cudaStream_t stream);
 
+// Tensor-core GEMM (gemm_tc.cu): shapes it covers, the launcher, and the count
+// of CTAs whose bounded pipeline wait gave up since the last read.
+bool gemm_tc_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,
+                           uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+cudaError_t read_and_clear_gemm_timeouts(unsigned int* count);
+
 // Largest K the GEMV accepts (x is staged in shared memory as fp32).
 constexpr int64_t kGemvMaxK = 49152;
 

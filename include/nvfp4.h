@@ -33,9 +33,11 @@
  *   - Arguments are validated on the host before anything is launched.  On
  *     failure nothing is enqueued, a status other than NVFP4_OK is returned and
  *     nvfp4_last_error() describes it.  No call aborts or throws.
- *   - Tensor pointers must be 16-byte aligned and scalar pointers (g, amax)
- *     4-byte aligned; leading dimensions are multiples of 8 elements.  K is a
- *     positive multiple of 16 (one scale per 16).
+ *   - Input tensor pointers (W, X, x, q, s) and the quantizer outputs q, s
+ *     must be 16-byte aligned, with leading dimensions ldw, ldx multiples of 8
+ *     elements; the BF16 outputs y, Y need 2-byte alignment and any ldy >= N;
+ *     scalar pointers (g, amax) need 4-byte alignment.  K is a positive
+ *     multiple of 16 (one scale per 16).
  *   - Calls on the same stream are ordered; calls on different streams that
  *     write the same buffers race.
  */
@@ -62,10 +64,11 @@ typedef enum nvfp4_status {
   NVFP4_OK = 0,
   NVFP4_ERR_INVALID_ARG = 1, /* null pointer, negative size, aliasing outputs */
   NVFP4_ERR_SHAPE = 2,       /* K not a positive multiple of 16, M/N < 0, size too large */
-  NVFP4_ERR_ALIGNMENT = 3,   /* pointer not 16-byte aligned, leading dim not a multiple of 8 */
+  NVFP4_ERR_ALIGNMENT = 3,   /* pointer under-aligned, leading dimension not a multiple of 8 */
   NVFP4_ERR_UNSUPPORTED = 4, /* current device is not compute capability 10.0 (B200) */
   NVFP4_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
-  NVFP4_ERR_WORKSPACE = 6    /* workspace missing or smaller than nvfp4_gemm_workspace_size() */
+  NVFP4_ERR_WORKSPACE = 6,   /* workspace missing or smaller than nvfp4_gemm_workspace_size() */
+  NVFP4_ERR_TIMEOUT = 7      /* a kernel's bounded pipeline wait gave up (see nvfp4_check_device_errors) */
 } nvfp4_status;
 
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
@@ -132,10 +135,11 @@ NVFP4_API nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uin
 /*
  * GEMM Y = X . W^T for M >= 1 rows of activations (32-user batched decode and
  * 512-token prefill of the model card "Qwen3.8-27B-NVFP4", "Measurements"),
- * same arithmetic as nvfp4_gemv per output.  M == 1 runs the GEMV.  M >= 2 runs
- * on the tensor cores (tcgen05, BF16 operands, fp32 accumulation in tensor
- * memory); the dequantized weights e2m1 * e4m3 are exact in BF16, g is applied
- * in fp32 in the epilogue.
+ * same arithmetic as nvfp4_gemv per output.  M == 1 runs the GEMV.  M >= 2 with
+ * K % 256 == 0 runs on the tensor cores (tcgen05, BF16 operands, fp32
+ * accumulation in tensor memory); the dequantized weights e2m1 * e4m3 are exact
+ * in BF16 and g is applied in fp32 in the epilogue.  Other K (<= 49152) run one
+ * GEMV per row of X.
  * workspace: device scratch of nvfp4_gemm_workspace_size(M, N, K) bytes, may be
  *   NULL when that size is 0.
  * Y must not overlap X, q or s.  M == 0 or N == 0 is a no-op.
@@ -147,6 +151,15 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t*
 
 /* Bytes of workspace nvfp4_gemm needs for this shape (0 if none). */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Diagnostic: every wait inside the tensor-core GEMM's pipeline is bounded (2 s
+ * of wall-clock time); a CTA that gives up records it in a device counter and
+ * finishes without hanging, leaving its outputs undefined.  This call reads and
+ * clears that counter for the current device (it waits for prior work on the
+ * legacy default stream) and returns NVFP4_ERR_TIMEOUT if it was non-zero.
+ */
+NVFP4_API nvfp4_status nvfp4_check_device_errors(void);
 
 #ifdef __cplusplus
 }

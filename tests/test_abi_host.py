@@ -42,6 +42,7 @@ def test_gemv_validation():
     assert nv.lib.nvfp4_gemv(None, A, A, A, A, 4, 64, None) == INVALID
     assert nv.lib.nvfp4_gemv(A + 8, A, A, A, A + 4096, 4, 64, None) == ALIGN
     assert nv.lib.nvfp4_gemv(A, A, A, A + 2, A + 4096, 4, 64, None) == ALIGN
+    assert nv.lib.nvfp4_gemv(A, A, A, A, A + 4097, 4, 64, None) == ALIGN
     assert nv.lib.nvfp4_gemv(A, A, A, A, A + 4096, 4, 49152 + 16, None) == SHAPE
     # y overlapping x
     assert nv.lib.nvfp4_gemv(A, A + 8192, A + 16384, A + 32768, A + 16, 4, 64, None) == INVALID
@@ -67,5 +68,6 @@ def test_amax_validation():
 def test_gemm_validation():
     assert nv.lib.nvfp4_gemm(A, 64, A, A, A, A, 64, 0, 64, 64, None, 0, None) == OK
     assert nv.lib.nvfp4_gemm(A, 32, A, A, A, A, 64, 4, 64, 64, None, 0, None) == INVALID  # ldx < K
-    assert nv.lib.nvfp4_gemm(A, 72, A, A, A, A, 68, 4, 64, 64, None, 0, None) == ALIGN   # ldy % 8
+    assert nv.lib.nvfp4_gemm(A, 68, A, A, A, A + 4096, 64, 4, 64, 64, None, 0, None) == ALIGN   # ldx % 8
+    assert nv.lib.nvfp4_gemm(A, 64, A, A, A, A + 4097, 64, 4, 64, 64, None, 0, None) == ALIGN   # odd Y
     assert nv.lib.nvfp4_gemm(A, 64, A, A, A, None, 64, 4, 64, 64, None, 0, None) == INVALID
