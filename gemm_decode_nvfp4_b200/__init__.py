@@ -4,7 +4,7 @@ Argument marshalling only: every entry point takes torch CUDA tensors, checks
 dtypes and shapes, and passes raw device pointers, leading dimensions and the
 current CUDA stream to the C ABI.  All arithmetic runs in the library's CUDA
 kernels; there is no CPU path.  Importing fails loudly if the library has not
-been built (``python -m gemm_decode_nvfp4_b200.build``).
+been built (``python gemm_decode_nvfp4_b200/build.py``).
 
 Layouts follow the NVFP4 format of the pages (imp docs/quantization.md, format
 table: packed nibbles, E4M3 micro-scales per 16, FP32 tensor scale):
@@ -21,6 +21,7 @@ import torch
 __all__ = [
     "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
+    "FLAG_STATIC_WEIGHTS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m gemm_decode_nvfp4_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python gemm_decode_nvfp4_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -40,10 +41,13 @@ lib.nvfp4_amax.argtypes = [_p, _i64, _i64, _i64, _p, _p]
 lib.nvfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p]
 lib.nvfp4_gemv.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _p]
 lib.nvfp4_gemm.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]
+lib.nvfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
+lib.nvfp4_gemm_ex.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
 lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
-for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_check_device_errors):
+for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
+           lib.nvfp4_check_device_errors):
     _f.restype = ctypes.c_int
 
 
@@ -127,9 +131,13 @@ def quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch.Ten
                                                 _ptr(g_out), _stream(stream)))
 
 
+FLAG_STATIC_WEIGHTS = 1
+
+
 def gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, y: torch.Tensor,
-         stream=None) -> None:
-    """y[N] = bf16(g * W_deq . x) for BF16 x [K] (or [1, K])."""
+         stream=None, static_weights: bool = False) -> None:
+    """y[N] = bf16(g * W_deq . x) for BF16 x [K] (or [1, K]).  static_weights: q, s, g
+    are not written by work still running on the stream (see NVFP4_FLAG_STATIC_WEIGHTS)."""
     _need(x, torch.bfloat16, "x")
     _need(q, torch.uint8, "q", 2)
     _need(s, torch.uint8, "s", 2)
@@ -140,7 +148,9 @@ def gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, y: 
         raise ValueError("x must hold K and y N contiguous elements")
     if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
-    _check("nvfp4_gemv", lib.nvfp4_gemv(_ptr(x), _ptr(q), _ptr(s), _ptr(g), _ptr(y), N, K, _stream(stream)))
+    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    _check("nvfp4_gemv_ex", lib.nvfp4_gemv_ex(_ptr(x), _ptr(q), _ptr(s), _ptr(g), _ptr(y), N, K, flags,
+                                              _stream(stream)))
 
 
 def gemm_workspace_size(M: int, N: int, K: int) -> int:
@@ -148,7 +158,7 @@ def gemm_workspace_size(M: int, N: int, K: int) -> int:
 
 
 def gemm(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, Y: torch.Tensor,
-         workspace: torch.Tensor | None = None, stream=None) -> None:
+         workspace: torch.Tensor | None = None, stream=None, static_weights: bool = False) -> None:
     """Y [M, N] = bf16(g * X . W_deq^T) for BF16 X [M, K]."""
     _need(X, torch.bfloat16, "X", 2)
     _need(q, torch.uint8, "q", 2)
@@ -165,8 +175,9 @@ def gemm(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, Y: 
     if workspace is not None:
         _need(workspace, torch.uint8, "workspace")
         ws_bytes = workspace.numel()
-    _check("nvfp4_gemm", lib.nvfp4_gemm(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0),
-                                        M, N, K, _ptr(workspace), ws_bytes, _stream(stream)))
+    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    _check("nvfp4_gemm_ex", lib.nvfp4_gemm_ex(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0),
+                                              M, N, K, _ptr(workspace), ws_bytes, flags, _stream(stream)))
 
 
 # ------------------------------------------------------ allocating helpers

@@ -1,6 +1,7 @@
 """Build libnvfp4.so (the C-ABI library of include/nvfp4.h) for sm_100a, in tree.
 
-Run ``python -m gemm_decode_nvfp4_b200.build`` (or call ``build()``).  nvcc
+Run ``python gemm_decode_nvfp4_b200/build.py`` (or call ``build()``; the
+package itself cannot be imported before the library exists).  nvcc
 cross-compiles without a GPU.  Each .cu is compiled to an object in
 ``_build/`` in parallel, then linked into ``gemm_decode_nvfp4_b200/libnvfp4.so``
 with the CUDA runtime linked statically.

@@ -33,6 +33,8 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return na && nb && pa < pb + nb && pb < pa + na;
 }
 
+constexpr uint32_t kKnownFlags = NVFP4_FLAG_STATIC_WEIGHTS;
+
 constexpr int kMaxDevices = 64;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
 int g_dev_sms[kMaxDevices];
@@ -144,6 +146,12 @@ nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw
 
 nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, nvfp4_stream_t stream) {
+  return nvfp4_gemv_ex(x, q, s, g, y, N, K, 0u, stream);
+}
+
+nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
+                           uint16_t* y, int64_t N, int64_t K, uint32_t flags, nvfp4_stream_t stream) {
+  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   nvfp4_status st = check_k(K);
   if (st != NVFP4_OK) return st;
   if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
@@ -162,7 +170,8 @@ nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
   int sms = 0;
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
-  cudaError_t e = nvfp4::launch_gemv(x, q, s, g, y, N, K, (cudaStream_t)stream);
+  cudaError_t e = nvfp4::launch_gemv(x, q, s, g, y, N, K, sms, (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0,
+                                     (cudaStream_t)stream);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "gemv launch");
 }
 
@@ -174,7 +183,14 @@ size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
                         const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  return nvfp4_gemm_ex(X, ldx, q, s, g, Y, ldy, M, N, K, workspace, workspace_bytes, 0u, stream);
+}
+
+nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                           const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           void* workspace, size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
   (void)workspace; (void)workspace_bytes;
+  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   nvfp4_status st = check_k(K);
   if (st != NVFP4_OK) return st;
   if (M < 0 || N < 0) return fail(NVFP4_ERR_SHAPE, "negative size M=%lld N=%lld", (long long)M, (long long)N);
@@ -191,7 +207,7 @@ nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const 
         overlaps(Y, yb, g, 4))
       return fail(NVFP4_ERR_INVALID_ARG, "Y must not overlap X, q, s or g");
   }
-  if (M == 1) return nvfp4_gemv(X, q, s, g, Y, N, K, stream);
+  if (M == 1) return nvfp4_gemv_ex(X, q, s, g, Y, N, K, flags, stream);
   int sms = 0;
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
@@ -204,17 +220,18 @@ nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const 
   if (K > nvfp4::kGemvMaxK) return fail(NVFP4_ERR_SHAPE, "K=%lld: the GEMM needs K %% 256 == 0 or K <= %lld",
                                         (long long)K, (long long)nvfp4::kGemvMaxK);
   for (int64_t m = 0; m < M; ++m) {
-    e = nvfp4::launch_gemv(X + m * ldx, q, s, g, Y + m * ldy, N, K, (cudaStream_t)stream);
+    e = nvfp4::launch_gemv(X + m * ldx, q, s, g, Y + m * ldy, N, K, sms, false, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "gemv launch");
   }
   return NVFP4_OK;
 }
 
 nvfp4_status nvfp4_check_device_errors(void) {
-  unsigned int n = 0;
+  unsigned int n = 0, m = 0;
   cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
+  if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_timeouts(&m);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error counter");
-  if (n) return fail(NVFP4_ERR_TIMEOUT, "%u tensor-core GEMM CTA(s) gave up on a pipeline wait", n);
+  if (n || m) return fail(NVFP4_ERR_TIMEOUT, "%u GEMM and %u GEMV CTA(s) gave up on a pipeline wait", n, m);
   return NVFP4_OK;
 }
 

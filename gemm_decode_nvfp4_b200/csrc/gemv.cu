@@ -33,24 +33,8 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 
-// c + lo(a)*lo(b) + hi(a)*hi(b) with a, b f16x2 pairs, in fp32 (products exact).
-__device__ __forceinline__ float fma2_f16_f32(uint32_t a2, uint32_t b2, float c) {
-  float d;
-  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"
-      "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.f16 t, al, bl, %3;\n\tfma.rn.f32.f16 %0, ah, bh, t;\n\t}"
-      : "=f"(d)
-      : "r"(a2), "r"(b2), "f"(c));
-  return d;
-}
 
-// floor(log2(v)) of a non-zero, finite BF16 magnitude given by its 15 low bits.
-__device__ __forceinline__ int bf16_ilogb(uint32_t a) {
-  return a >= 0x80u ? (int)(a >> 7) - 127 : (31 - __clz((int)a)) - 133;
-}
 
-// 2^k as fp32 for k in [-126, 127].
-__device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
 
 template <int R, int CB, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __restrict__ x,
@@ -261,7 +245,8 @@ cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const 
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
-                        uint16_t* y, int64_t N, int64_t K, cudaStream_t stream) {
+                        uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream) {
+  if (gemv_stream_supported(N, K)) return launch_gemv_stream(x, q, s, g, y, N, K, sms, static_weights, stream);
   if (K % 32 == 0) return launch<4, 16, 3>(x, q, s, g, y, (int)N, (int)K, stream);
   return launch<4, 8, 3>(x, q, s, g, y, (int)N, (int)K, stream);
 }

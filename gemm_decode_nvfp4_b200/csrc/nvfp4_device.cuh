@@ -89,4 +89,24 @@ __device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
   return v;
 }
 
+// c + lo(a)*lo(b) + hi(a)*hi(b) with a, b f16x2 pairs, in fp32: one
+// mixed-precision fma.rn.f32.f16 per product (products exact).
+__device__ __forceinline__ float fma2_f16_f32(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.f16 t, al, bl, %3;\n\tfma.rn.f32.f16 %0, ah, bh, t;\n\t}"
+      : "=f"(d)
+      : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+
+// floor(log2(v)) of a non-zero, finite BF16 magnitude given by its 15 low bits.
+__device__ __forceinline__ int bf16_ilogb(uint32_t a) {
+  return a >= 0x80u ? (int)(a >> 7) - 127 : (31 - __clz((int)a)) - 133;
+}
+
+// 2^k as fp32 for k in [-126, 127].
+__device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+
 }  // namespace nvfp4

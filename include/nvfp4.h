@@ -71,6 +71,17 @@ typedef enum nvfp4_status {
   NVFP4_ERR_TIMEOUT = 7      /* a kernel's bounded pipeline wait gave up (see nvfp4_check_device_errors) */
 } nvfp4_status;
 
+/*
+ * Flags of the *_ex entry points.
+ * NVFP4_FLAG_STATIC_WEIGHTS: q, s and g are not written by any work that is
+ *   still running on the stream when the call is made (model weights loaded
+ *   once).  The kernel may then start streaming them while the preceding
+ *   kernel on the stream is still finishing (programmatic dependent launch);
+ *   x / X are still read, and y / Y written, only after the preceding work has
+ *   completed.  Without the flag, every global access waits for it.
+ */
+#define NVFP4_FLAG_STATIC_WEIGHTS 1u
+
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 NVFP4_API int nvfp4_version(void);
 
@@ -132,6 +143,12 @@ NVFP4_API nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uin
                         const float* g, uint16_t* y, int64_t N, int64_t K,
                         nvfp4_stream_t stream);
 
+/* nvfp4_gemv with flags (NVFP4_FLAG_*); nvfp4_gemv(...) is this with flags 0.
+ * Unknown flag bits give NVFP4_ERR_INVALID_ARG. */
+NVFP4_API nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s,
+                                     const float* g, uint16_t* y, int64_t N, int64_t K,
+                                     uint32_t flags, nvfp4_stream_t stream);
+
 /*
  * GEMM Y = X . W^T for M >= 1 rows of activations (32-user batched decode and
  * 512-token prefill of the model card "Qwen3.8-27B-NVFP4", "Measurements"),
@@ -149,13 +166,20 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t*
                         int64_t K, void* workspace, size_t workspace_bytes,
                         nvfp4_stream_t stream);
 
+/* nvfp4_gemm with flags (NVFP4_FLAG_*); nvfp4_gemm(...) is this with flags 0. */
+NVFP4_API nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                                     const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                                     int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                     nvfp4_stream_t stream);
+
 /* Bytes of workspace nvfp4_gemm needs for this shape (0 if none). */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /*
- * Diagnostic: every wait inside the tensor-core GEMM's pipeline is bounded (2 s
- * of wall-clock time); a CTA that gives up records it in a device counter and
- * finishes without hanging, leaving its outputs undefined.  This call reads and
+ * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMM and
+ * the bulk-copy GEMV) is bounded (2 s of wall-clock time); a CTA that gives up
+ * records it in a device counter and finishes without hanging, leaving its
+ * outputs undefined.  This call reads and
  * clears that counter for the current device (it waits for prior work on the
  * legacy default stream) and returns NVFP4_ERR_TIMEOUT if it was non-zero.
  */

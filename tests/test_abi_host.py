@@ -71,3 +71,9 @@ def test_gemm_validation():
     assert nv.lib.nvfp4_gemm(A, 68, A, A, A, A + 4096, 64, 4, 64, 64, None, 0, None) == ALIGN   # ldx % 8
     assert nv.lib.nvfp4_gemm(A, 64, A, A, A, A + 4097, 64, 4, 64, 64, None, 0, None) == ALIGN   # odd Y
     assert nv.lib.nvfp4_gemm(A, 64, A, A, A, None, 64, 4, 64, 64, None, 0, None) == INVALID
+
+
+def test_unknown_flags_rejected():
+    assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 4, 64, 0x80, None) == INVALID
+    assert nv.lib.nvfp4_gemm_ex(A, 64, A, A, A, A + 4096, 64, 4, 64, 64, None, 0, 0x2, None) == INVALID
+    assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 0, 64, 1, None) == OK   # N == 0: no-op

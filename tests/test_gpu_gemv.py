@@ -146,3 +146,75 @@ def test_cuda_graph_replay(nv):
     graph.replay()
     torch.cuda.synchronize()
     assert_within_tolerance(y, y_ref[0], bound[0], "graph")
+
+
+@pytest.mark.parametrize("N,K", [(600, 5120), (130, 17408), (40, 1040)])
+@pytest.mark.parametrize("kind", ["wide", "tiny", "zero"])
+def test_x_dynamic_range_paths(nv, N, K, kind):
+    """x whose non-zero magnitudes span more than 2^32 takes the exact fp32
+    path; tiny-but-narrow x takes the scaled f16 path; all-zero x gives 0."""
+    q, s = workloads.random_codes(N, K, 13)
+    x = workloads.random_bf16((1, K), 14).float()
+    if kind == "wide":
+        x[0, 0] = 2.0 ** 100
+        x[0, 1] = -(2.0 ** -60)
+        x[0, 7] = 3.0e-30
+    elif kind == "tiny":
+        x = x * 2.0 ** -120          # BF16 subnormals and tiny normals, narrow range
+    else:
+        x = x * 0.0
+    x = x.to(torch.bfloat16)
+    y_ref, bound = oracle.linear(x, q.numpy(), s.numpy(), 0.75)
+    y = _run(nv, x, q.numpy(), s.numpy(), 0.75)
+    assert_within_tolerance(y, y_ref[0], bound[0], f"{kind} N={N} K={K}")
+    if kind == "zero":
+        assert not y.float().abs().sum().item()
+
+
+def test_static_weights_chain_in_graph(nv):
+    """Eight GEMVs back to back in one CUDA graph with static weights (programmatic
+    dependent launch), each feeding the next one's x: every output must match the
+    oracle run on the previous output."""
+    N = K = 5120
+    q, s, g = oracle.quantize(workloads.to_bf16(workloads.plain_weight_f32(N, K, 31)))
+    qd, sd = torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda()
+    gd = torch.tensor([float(g)], device="cuda")
+    x0 = workloads.random_bf16((K,), 32).cuda()
+    ys = [torch.empty((N,), dtype=torch.bfloat16, device="cuda") for _ in range(8)]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        nv.gemv(x0, qd, sd, gd, ys[0], static_weights=True)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        prev = x0
+        for y in ys:
+            nv.gemv(prev, qd, sd, gd, y, static_weights=True)
+            prev = y
+    graph.replay()
+    torch.cuda.synchronize()
+    prev = x0.cpu()
+    for i, y in enumerate(ys):
+        y_ref, bound = oracle.linear(prev.reshape(1, -1), q, s, g)
+        assert_within_tolerance(y, y_ref[0], bound[0], f"chain {i}")
+        prev = y.cpu()
+
+
+def test_quantize_then_gemv_same_stream(nv):
+    """The quantizer writes q, s, g and the GEMV (no static-weights flag) reads them
+    right after on the same stream: stream order must hold."""
+    N, K = 2048, 5120
+    w = workloads.random_bf16((N, K), 33, 0.02).cuda()
+    x = workloads.random_bf16((K,), 34).cuda()
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.empty((N, K // 16), dtype=torch.uint8, device="cuda")
+    g = torch.empty((1,), dtype=torch.float32, device="cuda")
+    y = torch.empty((N,), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        q.fill_(0); s.fill_(0)
+        nv.quantize(w, q, s, g)
+        nv.gemv(x, q, s, g, y)
+    torch.cuda.synchronize()
+    q_ref, s_ref, g_ref = oracle.quantize(w.cpu())
+    y_ref, bound = oracle.linear(x.cpu().reshape(1, -1), q_ref, s_ref, g_ref)
+    assert_within_tolerance(y, y_ref[0], bound[0], "quantize->gemv")
