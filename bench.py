@@ -177,18 +177,20 @@ def run_gpu(args):
     Y32 = [torch.empty((32, N), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
     X512 = workloads.activations(512, K, 4).to(dev)
     Y512 = torch.empty((512, N), dtype=torch.bfloat16, device=dev)
+    ws32 = torch.empty((max(1, nv.gemm_workspace_size(32, N, K)),), dtype=torch.uint8, device=dev)
+    ws512 = torch.empty((max(1, nv.gemm_workspace_size(512, N, K)),), dtype=torch.uint8, device=dev)
     wq_in = workloads.to_bf16(workloads.plain_weight_f32(N, K, 4)).to(dev)
     qq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
     sq = torch.empty((N, K // 16), dtype=torch.uint8, device=dev)
     gq = torch.empty((1,), dtype=torch.float32, device=dev)
 
-    gemm_ok = args.only != "gemv"
-    gemm_err = "not run (--only gemv)"
+    gemm_ok = args.only in ("all", "gemm_m32", "gemm_m512")
+    gemm_err = f"not run (--only {args.only})"
     try:
         if not gemm_ok:
             raise _Skip()
-        nv.gemm(X32, qs[0], ss[0], g0, Y32[0])
-        nv.gemm(X512, qs[0], ss[0], g0, Y512)
+        nv.gemm(X32, qs[0], ss[0], g0, Y32[0], workspace=ws32)
+        nv.gemm(X512, qs[0], ss[0], g0, Y512, workspace=ws512)
         torch.cuda.synchronize()
     except _Skip:
         pass
@@ -214,17 +216,19 @@ def run_gpu(args):
     rows.append(("gemv", gemv_all, copies, 1))
     rows.append(("gemv_ordered", gemv_ordered_all, copies, 1))
     rows.append(("quantize", quant_all, 1, 2))
-    if gemm_ok and args.only != "gemv":
+    if gemm_ok:
         def m32_all():
             for i in range(copies):
-                nv.gemm(X32, qs[i], ss[i], g0, Y32[i])
+                nv.gemm(X32, qs[i], ss[i], g0, Y32[i], workspace=ws32, static_weights=True)
 
         def m512_all():
             for i in range(copies):
-                nv.gemm(X512, qs[i], ss[i], g0, Y512)
+                nv.gemm(X512, qs[i], ss[i], g0, Y512, workspace=ws512, static_weights=True)
 
-        rows.append(("gemm_m32", m32_all, copies, 1))
-        rows.append(("gemm_m512", m512_all, copies, 1))
+        rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
+        rows.append(("gemm_m512", m512_all, copies, 2))
+    if args.only != "all":  # profiling runs: keep only the named row (plus the headline GEMV)
+        rows = [r for r in rows if r[0] in (args.only, "gemv")]
 
     graphs = {}
     with torch.cuda.stream(stream):
@@ -288,12 +292,15 @@ def run_gpu(args):
     kernels["gemv"] = {"us": per_launch_ms["gemv"] * 1e3, "GB/s": gemv_gbs, "frac_hbm": gemv_gbs / hbm,
                        "bytes": gb, "weight_bytes_per_token": N * K // 2 + N * K // 16,
                        "launch": "static weights: programmatic dependent launch between back-to-back GEMVs"}
-    go = gb / (per_launch_ms["gemv_ordered"] * 1e-3) / 1e9
-    kernels["gemv_ordered"] = {"us": per_launch_ms["gemv_ordered"] * 1e3, "GB/s": go, "frac_hbm": go / hbm,
-                               "launch": "no static-weights flag: all reads wait for the previous kernel"}
-    qb = quantize_bytes(N, K)
-    qgbs = qb / (per_launch_ms["quantize"] * 1e-3) / 1e9
-    kernels["quantize"] = {"us": per_launch_ms["quantize"] * 1e3, "GB/s": qgbs, "frac_hbm": qgbs / hbm, "bytes": qb}
+    if "gemv_ordered" in per_launch_ms:
+        go = gb / (per_launch_ms["gemv_ordered"] * 1e-3) / 1e9
+        kernels["gemv_ordered"] = {"us": per_launch_ms["gemv_ordered"] * 1e3, "GB/s": go, "frac_hbm": go / hbm,
+                                   "launch": "no static-weights flag: all reads wait for the previous kernel"}
+    if "quantize" in per_launch_ms:
+        qb = quantize_bytes(N, K)
+        qgbs = qb / (per_launch_ms["quantize"] * 1e-3) / 1e9
+        kernels["quantize"] = {"us": per_launch_ms["quantize"] * 1e3, "GB/s": qgbs, "frac_hbm": qgbs / hbm,
+                               "bytes": qb}
     for name, M in (("gemm_m32", 32), ("gemm_m512", 512)):
         if name in per_launch_ms:
             t = per_launch_ms[name] * 1e-3
@@ -302,7 +309,7 @@ def run_gpu(args):
             kernels[name] = {"us": t * 1e6, "TFLOP/s": fl / t / 1e12, "frac_bf16": fl / t / 1e12 / bf16_burst,
                              "GB/s": byt / t / 1e9, "frac_hbm": byt / t / 1e9 / hbm,
                              "weight_bytes_per_token": (N * K // 2 + N * K // 16) / M}
-        elif not gemm_ok:
+        elif not gemm_ok and args.only == "all":
             kernels[name] = {"unavailable": gemm_err}
 
     # ---- end to end through the public API with host buffers (decode GEMV):
@@ -448,8 +455,9 @@ def main():
     ap.add_argument("--copies", type=int, default=8, help="rotating weight copies per graph (L2 defeat)")
     ap.add_argument("--cpu-rows", type=int, default=17408)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "gemv"],
-                    help="gemv: time only the decode GEMV and quantizer rows (profiling runs)")
+    ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "gemm_m32",
+                                                      "gemm_m512"],
+                    help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -176,8 +176,8 @@ nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s
 }
 
 size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
-  (void)M; (void)N; (void)K;
-  return 0;
+  if (M < 2 || N < 1 || !nvfp4::gemm_tc_supported(M, N, K)) return 0;
+  return nvfp4::gemm_tc_workspace_bytes(M, K);
 }
 
 nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
@@ -189,7 +189,6 @@ nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const 
 nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
                            const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                            void* workspace, size_t workspace_bytes, uint32_t flags, nvfp4_stream_t stream) {
-  (void)workspace; (void)workspace_bytes;
   if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   nvfp4_status st = check_k(K);
   if (st != NVFP4_OK) return st;
@@ -213,7 +212,17 @@ nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, con
   if (st != NVFP4_OK) return st;
   cudaError_t e;
   if (nvfp4::gemm_tc_supported(M, N, K)) {
-    e = nvfp4::launch_gemm_tc(X, ldx, q, s, g, Y, ldy, M, N, K, (cudaStream_t)stream);
+    const size_t need = nvfp4::gemm_tc_workspace_bytes(M, K);
+    if (!workspace || workspace_bytes < need)
+      return fail(NVFP4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+    const size_t xb = (size_t)((M - 1) * ldx + K) * 2, yb = (size_t)((M - 1) * ldy + N) * 2;
+    if (overlaps(workspace, need, X, xb) || overlaps(workspace, need, Y, yb) ||
+        overlaps(workspace, need, q, (size_t)(N * K / 2)) || overlaps(workspace, need, s, (size_t)(N * K / 16)) ||
+        overlaps(workspace, need, g, 4))
+      return fail(NVFP4_ERR_INVALID_ARG, "workspace must not overlap X, Y, q, s or g");
+    e = nvfp4::launch_gemm_tc(X, ldx, q, s, g, Y, ldy, M, N, K, workspace, (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0,
+                              (cudaStream_t)stream);
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "tensor-core gemm launch");
   }
   // K not a multiple of 256: one decode GEMV per row of X (same arithmetic).

@@ -27,9 +27,13 @@ cudaError_t launch_gemv_stream(const uint16_t* x, const uint8_t* q, const uint8_
 
 // Tensor-core GEMM (gemm_tc.cu): shapes it covers, the launcher, and the count
 // of CTAs whose bounded pipeline wait gave up since the last read.
+// The workspace holds the per-row exponents and the f16 copy of X (see
+// gemm_tc_workspace_bytes); it must be 16-byte aligned.
 bool gemm_tc_supported(int64_t M, int64_t N, int64_t K);
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t K);
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,
-                           uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t stream);
+                           uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
+                           bool static_weights, cudaStream_t stream);
 cudaError_t read_and_clear_gemm_timeouts(unsigned int* count);
 cudaError_t read_and_clear_gemv_timeouts(unsigned int* count);
 

@@ -51,6 +51,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed
+// sleeps (up to the hint, in ns) instead of spinning, so waiting warps do not
+// take issue slots from working warps on the same scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_ns` of wall-clock time and returns false (the caller records the
 // error and stops issuing work).
@@ -119,6 +134,12 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// Same with f16 A and B (the operand types come from the instruction descriptor).
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  mma_bf16(d_tmem, a_desc, b_desc, idesc, accumulate);
+}
+
 // Arrive once on `bar` when all tcgen05.mma issued so far by this thread are done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -164,6 +185,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (1u << 7)                        // A format bf16
          | (1u << 10)                       // B format bf16
          | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// Instruction descriptor of kind::f16 with f16 A and B, fp32 accumulator,
+// both operands K-major, tile M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                          // D format fp32
+         | ((uint32_t)(N >> 3) << 17)       // N / 8  (A, B format 0 = f16)
          | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 

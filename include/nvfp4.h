@@ -153,12 +153,18 @@ NVFP4_API nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const 
  * GEMM Y = X . W^T for M >= 1 rows of activations (32-user batched decode and
  * 512-token prefill of the model card "Qwen3.8-27B-NVFP4", "Measurements"),
  * same arithmetic as nvfp4_gemv per output.  M == 1 runs the GEMV.  M >= 2 with
- * K % 256 == 0 runs on the tensor cores (tcgen05, BF16 operands, fp32
- * accumulation in tensor memory); the dequantized weights e2m1 * e4m3 are exact
- * in BF16 and g is applied in fp32 in the epilogue.  Other K (<= 49152) run one
+ * K % 256 == 0 runs on the tensor cores (tcgen05, fp32 accumulation in tensor
+ * memory): every product is exact, because the dequantized weights
+ * e2m1 * e4m3 are exact f16 values and each row of X is copied to f16 scaled
+ * by a power of two; rows whose non-zero magnitudes span more than 2^32 (or
+ * that are not finite) are recomputed exactly in fp32 on CUDA cores.  g and the
+ * row scale are applied in fp32 in the epilogue.  Other K (<= 49152) run one
  * GEMV per row of X.
- * workspace: device scratch of nvfp4_gemm_workspace_size(M, N, K) bytes, may be
- *   NULL when that size is 0.
+ * workspace: device scratch of at least nvfp4_gemm_workspace_size(M, N, K)
+ *   bytes, 16-byte aligned, not overlapping any argument (it receives the f16
+ *   copy of X and the row scales); may be NULL when that size is 0.  Too small
+ *   a workspace gives NVFP4_ERR_WORKSPACE.  Calls that share a workspace must
+ *   be ordered (one stream).
  * Y must not overlap X, q or s.  M == 0 or N == 0 is a no-op.
  */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,

@@ -18,7 +18,7 @@ def nv():
     return m
 
 
-def _run(nv, X_cpu, q_np, s_np, g, ldx=None, ldy=None):
+def _run(nv, X_cpu, q_np, s_np, g, ldx=None, ldy=None, static_weights=False):
     M, K = X_cpu.shape
     N = q_np.shape[0]
     ldx = ldx or K
@@ -32,8 +32,11 @@ def _run(nv, X_cpu, q_np, s_np, g, ldx=None, ldy=None):
     Ybuf, check = guarded_empty((M, ldy), torch.bfloat16)
     Ybuf.fill_(float("nan"))
     Y = Ybuf[:, :N]
-    nv.gemm(X, q, s, gd, Y)
+    n_ws = nv.gemm_workspace_size(M, N, K)
+    ws, check_ws = guarded_empty((max(n_ws, 1),), torch.uint8)
+    nv.gemm(X, q, s, gd, Y, workspace=ws if n_ws else None, static_weights=static_weights)
     check()
+    check_ws()
     assert nv.lib.nvfp4_check_device_errors() == 0
     if ldy > N:  # padding columns untouched
         assert torch.isnan(Ybuf[:, N:].float()).all()
@@ -127,14 +130,61 @@ def test_cuda_graph_replay(nv):
     Xd, qd, sd = X.cuda(), q.cuda(), s.cuda()
     gd = torch.tensor([0.125], device="cuda")
     Y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((nv.gemm_workspace_size(M, N, K),), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
-        nv.gemm(Xd, qd, sd, gd, Y)
+        nv.gemm(Xd, qd, sd, gd, Y, workspace=ws, static_weights=True)
     stream.synchronize()
     Y.zero_()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        nv.gemm(Xd, qd, sd, gd, Y)
+        nv.gemm(Xd, qd, sd, gd, Y, workspace=ws, static_weights=True)
     graph.replay()
     torch.cuda.synchronize()
     assert_within_tolerance(Y, y_ref, bound, "graph")
+
+
+@pytest.mark.parametrize("M", [5, 40, 300])
+def test_wide_range_rows_recomputed_exactly(nv, M):
+    """Rows of X whose non-zero magnitudes span more than 2^32 (and rows of huge
+    or tiny scale) must still match the oracle: the wide ones are recomputed in
+    fp32 on CUDA cores, the others go through the scaled f16 MMA."""
+    N, K = 256, 1024
+    q, s = workloads.random_codes(N, K, 40 + M)
+    X = workloads.random_bf16((M, K), 41 + M).float()
+    X[0, 3] = 2.0 ** 90            # wide row
+    X[0, 9] = 2.0 ** -70
+    X[M - 1] *= 2.0 ** -125        # tiny but narrow row
+    if M > 2:
+        X[1] *= 2.0 ** 100         # huge but narrow row
+        X[2, :] = 0.0              # all-zero row
+    X = X.to(torch.bfloat16)
+    y_ref, bound = oracle.linear(X, q.numpy(), s.numpy(), 0.3)
+    Y = _run(nv, X, q.numpy(), s.numpy(), 0.3)
+    assert_within_tolerance(Y, y_ref, bound, f"wide rows M={M}")
+
+
+def test_static_weights_flag_matches(nv):
+    M, N, K = 64, 384, 2048
+    q, s = workloads.random_codes(N, K, 50)
+    X = workloads.random_bf16((M, K), 51)
+    y_ref, bound = oracle.linear(X, q.numpy(), s.numpy(), 0.5)
+    Y = _run(nv, X, q.numpy(), s.numpy(), 0.5, static_weights=True)
+    assert_within_tolerance(Y, y_ref, bound, "static weights")
+
+
+def test_workspace_too_small_is_an_error(nv):
+    M, N, K = 32, 128, 256
+    X = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((N, K // 16), dtype=torch.uint8, device="cuda")
+    g = torch.ones((1,), device="cuda")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    need = nv.gemm_workspace_size(M, N, K)
+    assert need > 0
+    small = torch.empty((need - 16,), dtype=torch.uint8, device="cuda")
+    with pytest.raises(nv.Nvfp4Error) as ei:
+        nv.gemm(X, q, s, g, Y, workspace=small)
+    assert ei.value.status == 6
+    with pytest.raises(nv.Nvfp4Error):
+        nv.gemm(X, q, s, g, Y)
