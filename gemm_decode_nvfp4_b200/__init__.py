@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
-    "FLAG_STATIC_WEIGHTS",
+    "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -43,11 +43,12 @@ lib.nvfp4_gemv.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _p]
 lib.nvfp4_gemm.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]
 lib.nvfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_ex.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, ctypes.c_uint32, _p]
+lib.nvfp4_gemm_noalloc.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
 lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
 for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
-           lib.nvfp4_check_device_errors):
+           lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors):
     _f.restype = ctypes.c_int
 
 
@@ -178,6 +179,39 @@ def gemm(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, Y: 
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
     _check("nvfp4_gemm_ex", lib.nvfp4_gemm_ex(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0),
                                               M, N, K, _ptr(workspace), ws_bytes, flags, _stream(stream)))
+
+
+def _header_constant(name: str) -> int:
+    with open(HEADER_PATH) as f:
+        m = re.search(r"#define\s+" + name + r"\s+\(\(\(size_t\)(\d+) << (\d+)\) \+ (\d+)\)", f.read())
+    if not m:
+        raise ImportError(f"{name} not found in {HEADER_PATH}")
+    return (int(m.group(1)) << int(m.group(2))) + int(m.group(3))
+
+
+# Bytes of the scratch array built into the library for gemm_noalloc.
+GEMM_NOALLOC_SCRATCH_BYTES = _header_constant("NVFP4_GEMM_NOALLOC_SCRATCH_BYTES")
+
+
+def gemm_noalloc(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, Y: torch.Tensor,
+                 stream=None, static_weights: bool = False) -> None:
+    """gemm() with the library's built-in scratch instead of a workspace
+    (nvfp4_gemm_noalloc): allocates nothing, for callers that cannot.  Calls on
+    one device share the scratch and must be ordered (one stream)."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    _need(g, torch.float32, "g")
+    _need(Y, torch.bfloat16, "Y", 2)
+    M, K = X.shape
+    N = q.shape[0]
+    if q.shape[1] * 2 != K or Y.shape != (M, N):
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
+    if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
+        raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
+    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    _check("nvfp4_gemm_noalloc", lib.nvfp4_gemm_noalloc(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y),
+                                                        Y.stride(0), M, N, K, flags, _stream(stream)))
 
 
 # ------------------------------------------------------ allocating helpers

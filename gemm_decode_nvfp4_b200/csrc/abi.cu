@@ -69,6 +69,16 @@ nvfp4_status check_k(int64_t K) {
 
 }  // namespace
 
+nvfp4_status nvfp4::report_error(nvfp4_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+nvfp4_status nvfp4::report_cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+
 extern "C" {
 
 int nvfp4_version(void) { return 100; }

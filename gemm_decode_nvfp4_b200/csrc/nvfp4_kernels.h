@@ -7,6 +7,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "nvfp4.h"
+
 namespace nvfp4 {
 
 cudaError_t launch_amax(const uint16_t* w, int64_t rows, int64_t cols, int64_t ldw, float* amax,
@@ -36,6 +38,11 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, con
                            bool static_weights, cudaStream_t stream);
 cudaError_t read_and_clear_gemm_timeouts(unsigned int* count);
 cudaError_t read_and_clear_gemv_timeouts(unsigned int* count);
+
+// Record a message for nvfp4_last_error() on this thread and return st (or
+// NVFP4_ERR_CUDA for a CUDA error), for entry points defined outside abi.cu.
+nvfp4_status report_error(nvfp4_status st, const char* fmt, ...);
+nvfp4_status report_cuda_error(cudaError_t e, const char* what);
 
 // Largest K the GEMV accepts (x is staged in shared memory as fp32).
 constexpr int64_t kGemvMaxK = 49152;

@@ -181,6 +181,30 @@ NVFP4_API nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8
 /* Bytes of workspace nvfp4_gemm needs for this shape (0 if none). */
 NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
+/* Size of the scratch array built into the library for nvfp4_gemm_noalloc. */
+#define NVFP4_GEMM_NOALLOC_SCRATCH_BYTES (((size_t)8 << 20) + 4096)
+
+/*
+ * nvfp4_gemm_ex without a workspace argument: the scratch comes from an
+ * 8 MiB + 4 KiB array compiled into the library (one per device), so the call
+ * allocates nothing.  The pages have no counterpart of this entry point; it
+ * is for callers that cannot allocate device memory (no allocator of their
+ * own, or one that is closed while a step runs).
+ * Arguments, layouts, flags and results are those of nvfp4_gemm_ex.
+ * Limit: shapes whose nvfp4_gemm_workspace_size(M, N, K) exceeds
+ *   NVFP4_GEMM_NOALLOC_SCRATCH_BYTES are rejected with NVFP4_ERR_WORKSPACE
+ *   and launch nothing; every shape with M <= 1024 and M * K <= 2^22 fits
+ *   (e.g. M = 512, K = 8192).
+ * Set-up: the first call on each device (with that device current) looks up
+ *   the array's device address; make it before any stream capture begins.
+ * Sharing: every call on a device uses the same array, which keeps what the
+ *   last call wrote (nothing in it needs to start at zero).  Calls whose work
+ *   overlaps on the GPU race on it: order them (e.g. one stream).
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                                          const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                                          int64_t K, uint32_t flags, nvfp4_stream_t stream);
+
 /*
  * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMM and
  * the bulk-copy GEMV) is bounded (2 s of wall-clock time); a CTA that gives up

@@ -1,0 +1,125 @@
+"""nvfp4_gemm_noalloc (the GEMM with the library's built-in scratch) against
+nvfp4_gemm with a caller workspace, within the tests' tolerance
+|y - y_ref| <= 1e-3 * sum|w x| + 1e-2 * |y_ref|, on consecutive calls that
+share the scratch.  Collected last so that it also runs after every other
+test has used the library; it needs no state from them."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+
+@pytest.fixture(scope="module")
+def nv():
+    import gemm_decode_nvfp4_b200 as m
+    return m
+
+
+def _device_inputs(X_cpu, q_np, s_np, g):
+    X = X_cpu.cuda()
+    q = torch.from_numpy(np.ascontiguousarray(q_np)).cuda()
+    s = torch.from_numpy(np.ascontiguousarray(s_np)).cuda()
+    gd = torch.tensor([float(np.float32(g))], dtype=torch.float32, device="cuda")
+    return X, q, s, gd
+
+
+def _with_workspace(nv, X, q, s, gd):
+    M, N, K = X.shape[0], q.shape[0], X.shape[1]
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    n_ws = nv.gemm_workspace_size(M, N, K)
+    ws = torch.empty((n_ws,), dtype=torch.uint8, device="cuda") if n_ws else None
+    nv.gemm(X, q, s, gd, Y, workspace=ws)
+    return Y
+
+
+def _noalloc_raw(nv, X, q, s, gd, Y):
+    """Straight through the C ABI (ctypes), not the Python wrapper."""
+    M, N, K = X.shape[0], q.shape[0], X.shape[1]
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return nv.lib.nvfp4_gemm_noalloc(ctypes.c_void_p(X.data_ptr()), X.stride(0), ctypes.c_void_p(q.data_ptr()),
+                                     ctypes.c_void_p(s.data_ptr()), ctypes.c_void_p(gd.data_ptr()),
+                                     ctypes.c_void_p(Y.data_ptr()), Y.stride(0), M, N, K, 0, stream)
+
+
+def _check_pair(nv, X_cpu, q_np, s_np, g, what):
+    X, q, s, gd = _device_inputs(X_cpu, q_np, s_np, g)
+    Y_ref = _with_workspace(nv, X, q, s, gd)
+    Y = torch.full_like(Y_ref, float("nan"))
+    assert _noalloc_raw(nv, X, q, s, gd, Y) == 0, nv.lib.nvfp4_last_error().decode()
+    torch.cuda.synchronize()
+    assert nv.lib.nvfp4_check_device_errors() == 0
+    _, bound = oracle.linear(X_cpu, q_np, s_np, g)
+    y_ref = Y_ref.float().cpu().double().numpy()
+    y = Y.float().cpu().double().numpy()
+    tol = oracle.tolerance(y_ref, bound)
+    err = np.abs(y - y_ref)
+    assert np.all(err <= tol), f"{what}: {int(np.sum(~(err <= tol)))} outputs out of tolerance"
+    return Y, Y_ref
+
+
+@pytest.mark.gpu
+def test_two_calls_in_a_row_match_gemm(nv):
+    """Two consecutive calls of different shapes, then two of the same shape
+    with different X: each output agrees with nvfp4_gemm on a fresh workspace,
+    whatever the previous call left in the shared scratch."""
+    cases = [(64, 384, 1024, 11), (32, 384, 512, 12), (48, 256, 768, 13), (48, 256, 768, 14)]
+    for M, N, K, seed in cases:
+        q, s = workloads.random_codes(N, K, seed)
+        X = workloads.random_bf16((M, K), 100 + seed)
+        _check_pair(nv, X, q.numpy(), s.numpy(), 0.0123, f"M={M} N={N} K={K} seed={seed}")
+
+
+@pytest.mark.gpu
+def test_prefill_width_and_wide_rows(nv):
+    """M=512 at the prefill K=5120 (the largest shape the bench times, inside
+    the scratch limit), with one row whose range forces the exact CUDA-core
+    recompute; called twice in a row."""
+    M, N, K = 512, 256, 5120
+    q, s = workloads.random_codes(N, K, 21)
+    for rep in range(2):
+        X = workloads.random_bf16((M, K), 200 + rep)
+        X[7, 0] = 2.0 ** 60
+        X[7, 1] = 2.0 ** -60
+        _check_pair(nv, X, q.numpy(), s.numpy(), 0.003, f"prefill rep {rep}")
+
+
+@pytest.mark.gpu
+def test_paths_without_scratch(nv):
+    """M == 1 (the GEMV) and K % 256 != 0 (one GEMV per row) need no scratch;
+    the entry point still matches nvfp4_gemm there."""
+    for M, N, K, seed in [(1, 300, 1024, 31), (5, 200, 272, 32)]:
+        q, s = workloads.random_codes(N, K, seed)
+        X = workloads.random_bf16((M, K), seed + 1)
+        _check_pair(nv, X, q.numpy(), s.numpy(), 0.02, f"M={M} K={K}")
+
+
+@pytest.mark.gpu
+def test_oversize_is_rejected_on_gpu(nv):
+    """A shape whose scratch exceeds the built-in array returns
+    NVFP4_ERR_WORKSPACE and launches nothing (Y keeps its contents)."""
+    M, N, K = 1024, 128, 8192
+    assert nv.gemm_workspace_size(M, N, K) > nv.GEMM_NOALLOC_SCRATCH_BYTES
+    q, s = workloads.random_codes(N, K, 41)
+    X = workloads.random_bf16((M, K), 42)
+    Xd, qd, sd, gd = _device_inputs(X, q.numpy(), s.numpy(), 0.5)
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert _noalloc_raw(nv, Xd, qd, sd, gd, Y) == 6
+    assert b"built-in scratch" in nv.lib.nvfp4_last_error()
+    torch.cuda.synchronize()
+    assert torch.isnan(Y.float()).all()
+
+
+def test_oversize_is_rejected_on_host(nv):
+    """The size limit is checked on the host before anything touches a device."""
+    null = ctypes.c_void_p(0)
+    M, N, K = 4096, 64, 4096
+    st = nv.lib.nvfp4_gemm_noalloc(null, K, null, null, null, null, N, M, N, K, 0, null)
+    assert st == 6
+    assert b"built-in scratch" in nv.lib.nvfp4_last_error()
+    # The largest shapes the header promises fit within the array.
+    for M, K in [(1024, 4096), (512, 8192), (2, 1 << 21)]:
+        assert nv.gemm_workspace_size(M, 128, K) <= nv.GEMM_NOALLOC_SCRATCH_BYTES
