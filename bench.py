@@ -70,18 +70,30 @@ def kernel_source_hash(files) -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel: str, src_files):
-    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it was
-    taken on the current source of that kernel; else None."""
+# Sources each timed row's kernels are built from: a committed traffic figure
+# counts only while these files are unchanged since the ncu capture.
+_CSRC = "gemm_decode_nvfp4_b200/csrc/"
+KERNEL_SOURCES = {
+    "gemv": [_CSRC + "gemv_stream.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
+    "quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
+    "gemm_m32": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
+    "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
+}
+
+
+def traffic_from_profiles(row: str):
+    """DRAM bytes (read + write) per call of a timed row from the committed ncu
+    summary profiles/traffic.json, if it was taken on the current source of that
+    row's kernels; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or row not in KERNEL_SOURCES:
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel)
-    if not e or e.get("source_hash") != kernel_source_hash(src_files):
+    e = d.get(row)
+    if not e or e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[row]):
         return None
-    return e.get("dram_bytes_per_launch")
+    return e.get("dram_bytes_per_call")
 
 
 # ------------------------------------------------------------ clock sampler
@@ -341,8 +353,10 @@ def run_gpu(args):
     for name, _, n_launch, n_kern in rows:
         launches += args.steps * n_launch * n_kern
 
-    traffic = traffic_from_profiles("gemv", ["gemm_decode_nvfp4_b200/csrc/gemv.cu",
-                                             "gemm_decode_nvfp4_b200/csrc/nvfp4_device.cuh"])
+    for name in kernels:
+        if "us" in kernels[name]:
+            kernels[name]["traffic"] = traffic_from_profiles(name)
+    traffic = kernels["gemv"]["traffic"]
     out = None
     if rank == 0:
         out = {
