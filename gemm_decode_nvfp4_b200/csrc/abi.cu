@@ -180,13 +180,16 @@ nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s
   int sms = 0;
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
-  cudaError_t e = nvfp4::launch_gemv(x, q, s, g, y, N, K, sms, (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0,
-                                     (cudaStream_t)stream);
+  const bool static_w = (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0;
+  cudaError_t e;
+  e = nvfp4::launch_gemv(x, q, s, g, y, N, K, sms, static_w, (cudaStream_t)stream);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "gemv launch");
 }
 
 size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
-  if (M < 2 || N < 1 || !nvfp4::gemm_tc_supported(M, N, K)) return 0;
+  if (M < 2 || N < 1) return 0;
+  if (M <= 64 && nvfp4::gemm_small_supported(M, N, K)) return nvfp4::gemm_small_workspace_bytes(M, K);
+  if (!nvfp4::gemm_tc_supported(M, N, K)) return 0;
   return nvfp4::gemm_tc_workspace_bytes(M, K);
 }
 
@@ -221,8 +224,9 @@ nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, con
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
   cudaError_t e;
-  if (nvfp4::gemm_tc_supported(M, N, K)) {
-    const size_t need = nvfp4::gemm_tc_workspace_bytes(M, K);
+  const bool static_w = (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0;
+  auto check_workspace = [&](size_t need) -> nvfp4_status {
+    if (need == 0) return NVFP4_OK;
     if (!workspace || workspace_bytes < need)
       return fail(NVFP4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
     if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
@@ -231,8 +235,20 @@ nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, con
         overlaps(workspace, need, q, (size_t)(N * K / 2)) || overlaps(workspace, need, s, (size_t)(N * K / 16)) ||
         overlaps(workspace, need, g, 4))
       return fail(NVFP4_ERR_INVALID_ARG, "workspace must not overlap X, Y, q, s or g");
-    e = nvfp4::launch_gemm_tc(X, ldx, q, s, g, Y, ldy, M, N, K, workspace, (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0,
-                              (cudaStream_t)stream);
+    return NVFP4_OK;
+  };
+  if (M <= 64 && nvfp4::gemm_small_supported(M, N, K)) {
+    const size_t need = nvfp4::gemm_small_workspace_bytes(M, K);
+    st = check_workspace(need);
+    if (st != NVFP4_OK) return st;
+    e = nvfp4::launch_gemm_small(X, ldx, q, s, g, Y, ldy, M, N, K, need ? workspace : nullptr, static_w,
+                                 (cudaStream_t)stream);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "tensor-core gemm launch");
+  }
+  if (nvfp4::gemm_tc_supported(M, N, K)) {
+    st = check_workspace(nvfp4::gemm_tc_workspace_bytes(M, K));
+    if (st != NVFP4_OK) return st;
+    e = nvfp4::launch_gemm_tc(X, ldx, q, s, g, Y, ldy, M, N, K, workspace, static_w, (cudaStream_t)stream);
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "tensor-core gemm launch");
   }
   // K not a multiple of 256: one decode GEMV per row of X (same arithmetic).
@@ -246,11 +262,13 @@ nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, con
 }
 
 nvfp4_status nvfp4_check_device_errors(void) {
-  unsigned int n = 0, m = 0;
+  unsigned int n = 0, m = 0, k = 0;
   cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_timeouts(&m);
+  if (e == cudaSuccess) e = nvfp4::read_and_clear_small_timeouts(&k);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error counter");
-  if (n || m) return fail(NVFP4_ERR_TIMEOUT, "%u GEMM and %u GEMV CTA(s) gave up on a pipeline wait", n, m);
+  if (n || m || k)
+    return fail(NVFP4_ERR_TIMEOUT, "%u GEMM, %u small-M GEMM and %u GEMV CTA(s) gave up on a pipeline wait", n, k, m);
   return NVFP4_OK;
 }
 

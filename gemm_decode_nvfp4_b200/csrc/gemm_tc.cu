@@ -559,18 +559,29 @@ bool gemm_tc_supported(int64_t M, int64_t N, int64_t K) {
          M <= ((int64_t)1 << 31) - 512;
 }
 
-size_t gemm_tc_workspace_bytes(int64_t M, int64_t K) { return align16((size_t)M * 4) + (size_t)M * K * 2; }
+size_t gemm_prep_workspace_bytes(int64_t M, int64_t K) { return align16((size_t)M * 4) + (size_t)M * K * 2; }
+
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t K) { return gemm_prep_workspace_bytes(M, K); }
+
+cudaError_t launch_gemm_prep(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, void* workspace, int** info_out,
+                             uint16_t** xh_out, cudaStream_t stream) {
+  int* info = reinterpret_cast<int*>(workspace);
+  uint16_t* Xh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(workspace) + align16((size_t)M * 4));
+  *info_out = info;
+  *xh_out = Xh;
+  const uint16_t* xp = X;
+  int kk = (int)K;
+  void* args[] = {(void*)&xp, &ldx, &kk, (void*)&info, (void*)&Xh};
+  return launch_pdl((const void*)prep_x_kernel, dim3((unsigned)M), dim3(128), 0, stream, args);
+}
 
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,
                            uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
                            bool static_weights, cudaStream_t stream) {
-  int* info = reinterpret_cast<int*>(workspace);
-  uint16_t* Xh = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(workspace) + align16((size_t)M * 4));
+  int* info = nullptr;
+  uint16_t* Xh = nullptr;
   {
-    const uint16_t* xp = X;
-    int kk = (int)K;
-    void* args[] = {(void*)&xp, &ldx, &kk, (void*)&info, (void*)&Xh};
-    cudaError_t e = launch_pdl((const void*)prep_x_kernel, dim3((unsigned)M), dim3(128), 0, stream, args);
+    cudaError_t e = launch_gemm_prep(X, ldx, M, K, workspace, &info, &Xh, stream);
     if (e != cudaSuccess) return e;
   }
   const int m = (int)M, n = (int)N, k = (int)K;

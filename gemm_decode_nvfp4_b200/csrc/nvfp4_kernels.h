@@ -37,6 +37,22 @@ cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, con
                            uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
                            bool static_weights, cudaStream_t stream);
 cudaError_t read_and_clear_gemm_timeouts(unsigned int* count);
+
+// X pre-pass of the tensor-core GEMMs (gemm_tc.cu): per-row exponents and the
+// exact f16 copy of X, written into `workspace` (gemm_prep_workspace_bytes).
+size_t gemm_prep_workspace_bytes(int64_t M, int64_t K);
+cudaError_t launch_gemm_prep(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, void* workspace, int** info,
+                             uint16_t** xh, cudaStream_t stream);
+
+// Decode GEMV and small-M GEMM (gemm_small.cu, 1 <= M <= 64, K % 256 == 0):
+// dequantized weights in tensor memory.  M <= 8 needs no workspace (the kernel
+// converts X itself); larger M use the X pre-pass.
+bool gemm_small_supported(int64_t M, int64_t N, int64_t K);
+size_t gemm_small_workspace_bytes(int64_t M, int64_t K);
+cudaError_t launch_gemm_small(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,
+                              uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
+                              bool static_weights, cudaStream_t stream);
+cudaError_t read_and_clear_small_timeouts(unsigned int* count);
 cudaError_t read_and_clear_gemv_timeouts(unsigned int* count);
 
 // Record a message for nvfp4_last_error() on this thread and return st (or
