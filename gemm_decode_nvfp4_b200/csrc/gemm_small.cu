@@ -64,6 +64,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kWideRow = -(1 << 30);
 constexpr uint32_t kTmemCols = 512;
 constexpr int kConvMaxM = 8;
+constexpr int kEpiBar = 2;       // named barrier of the 16 dequantization warps (1 is the range scan)
 
 struct SmallBars {
   uint64_t wfull[16], wempty[16];  // weight stage landed / read by the 16 dequant warps
@@ -73,6 +74,7 @@ struct SmallBars {
   uint32_t tmem_addr;
   volatile int err;
   uint32_t xmax[kConvMaxM], xmin[kConvMaxM];  // per-row |x| range as BF16 bits (M <= 8 path)
+  int info[64];                    // the tile's row exponents (or kWideRow), staged for the epilogue
 };
 
 template <int BNT, bool CONV>
@@ -120,6 +122,19 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Sma
     atomicAdd(&g_small_wait_timeouts, 1u);
   }
   return false;
+}
+
+// OR of `v` over the `count` threads that meet at named barrier `id` (a
+// barrier: shared-memory writes before it are visible to all after it).
+__device__ __forceinline__ bool group_any(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -458,6 +473,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // ------------------------------------------------------------ epilogue
       if (static_weights) asm volatile("griddepcontrol.wait;" ::: "memory");  // row info and Y
+      // stage the tile's row info once and find out whether any row needs the
+      // exact recompute
+      bool wide_here = false;
+      for (int i = dw * 32 + lane; i < BNT; i += kDeqWarps * 32) {
+        const int m = m0 + i;
+        const int e = m >= M ? 0 : (CONV ? row_exponent(bars->xmax[m], bars->xmin[m]) : __ldg(info + m));
+        bars->info[i] = e;
+        wide_here |= e == kWideRow;
+      }
+      const bool any_wide = group_any(kEpiBar, kDeqWarps * 32, wide_here);
       const bool acc_ready = __all_sync(0xFFFFFFFFu, wait_or_fail(&bars->tmem_full, 0, bars));
       const float gv = *g;
       if (acc_ready) {
@@ -479,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 16; ++j) {
               const int m = m0 + 16 * grp + j;
               if (m < M) {
-                const int e = CONV ? row_exponent(bars->xmax[m], bars->xmin[m]) : __ldg(info + m);
+                const int e = bars->info[16 * grp + j];
                 if (e != kWideRow) {
                   const __nv_bfloat16 o = __float2bfloat16_rn((acc[j] * gv) * pow2f(-e));
                   Y[(int64_t)m * ldy + n] = *reinterpret_cast<const uint16_t*>(&o);
@@ -493,11 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // row (quarters of K), combined with two shuffles
       const int t = dw * 32 + lane;
       const int row = n0 + (t >> 2), part = t & 3;
-      for (int mi = 0; mi < BNT; ++mi) {
+      for (int mi = 0; mi < BNT && any_wide; ++mi) {
         const int m = m0 + mi;
         if (m >= M) break;
-        const int e = CONV ? row_exponent(bars->xmax[m], bars->xmin[m]) : __ldg(info + m);
-        if (e != kWideRow) continue;
+        if (bars->info[mi] != kWideRow) continue;
         float p = 0.0f;
         if (row < N) p = exact_dot(q, s, row, K, X + (int64_t)m * ldx, part * (K / 4), (part + 1) * (K / 4));
         p += __shfl_xor_sync(0xFFFFFFFFu, p, 1);

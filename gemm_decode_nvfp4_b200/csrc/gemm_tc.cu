@@ -69,6 +69,7 @@ struct Bars {
   uint64_t tmem_full; // last MMA finished
   uint32_t tmem_addr;
   volatile int err;
+  int info[512];      // the tile's row exponents (or kWideRow), staged for the epilogue
 };
 
 template <int BN, int NSUB>
@@ -83,8 +84,8 @@ struct Cfg {
   // A tiles are produced on chip and X' comes from L2; the weights come from
   // HBM with microseconds of latency under load, so the shared memory left
   // after the A and X' rings goes to a deep weight ring.
-  static constexpr int kBudget = 206 * 1024;
-  static constexpr int kStages = kBNT >= 256 ? 2 : 3;                    // A ring
+  static constexpr int kBudget = 218 * 1024;
+  static constexpr int kStages = kBNT >= 512 ? 3 : (kBNT >= 256 ? 2 : 3);  // A ring
   static constexpr int kXStages = kXG == 4 ? 3 : (kBNT >= 256 ? 2 : 3);  // X' ring
   static constexpr int kFixed = kStages * kABytes + kXStages * kXBytes;
   static constexpr int kWFit = (kBudget - kFixed) / (kWBytes + kSBytes);
@@ -131,6 +132,19 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
 __device__ __forceinline__ uint4 dequant8_f16(uint32_t word, uint32_t s2) {
   return make_uint4(hmul2(e2m1x2_byte_to_f16x2<0>(word), s2), hmul2(e2m1x2_byte_to_f16x2<1>(word), s2),
                     hmul2(e2m1x2_byte_to_f16x2<2>(word), s2), hmul2(e2m1x2_byte_to_f16x2<3>(word), s2));
+}
+
+// OR of `v` over the `count` threads that meet at named barrier `id` (a
+// barrier: shared-memory writes before it are visible to all after it).
+__device__ __forceinline__ bool group_any(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 // 2^k as fp32 for k in [-149, 127] (subnormal below -126).
@@ -410,6 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ptx::mbar_arrive(&bars->wempty[ws]);
     }
     if (static_weights) asm volatile("griddepcontrol.wait;" ::: "memory");  // info and Y
+    // stage the tile's row info once (the epilogue reads it per element) and
+    // find out whether any row needs the exact recompute
+    bool wide_here = false;
+    for (int i = t; i < BNT; i += kDeqWarps * 32) {
+      const int e = m0 + i < M ? __ldg(info + m0 + i) : 0;
+      bars->info[i] = e;
+      wide_here |= e == kWideRow;
+    }
+    const bool any_wide = group_any(1, kDeqWarps * 32, wide_here);
     // epilogue: TMEM lane (32 * (warp % 4) + lane) holds weight row n; columns are m.
     const bool acc_ready = __all_sync(0xFFFFFFFFu, wait_or_fail(&bars->tmem_full, 0, bars));
     if (acc_ready) {
@@ -433,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) {
               const int m = m0 + c0 + j;
               if (c0 + j < c_begin + kColsPerWarp && m < M) {
-                const int e = __ldg(info + m);
+                const int e = bars->info[c0 + j];
                 if (e != kWideRow) {
                   const float v = (__uint_as_float(rr[j]) * gv) * pow2f(-e);
                   const __nv_bfloat16 o = __float2bfloat16_rn(v);
@@ -448,10 +471,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rows of X outside the exact f16 window: exact fp32 dot on CUDA cores,
     // two threads per weight row (halves of K), combined with one shuffle
     const float gv = *g;
-    for (int mi = 0; mi < BNT; ++mi) {
+    for (int mi = 0; mi < BNT && any_wide; ++mi) {
       const int m = m0 + mi;
       if (m >= M) break;
-      if (__ldg(info + m) != kWideRow) continue;
+      if (bars->info[mi] != kWideRow) continue;
       float part = 0.0f;
       if (row_ok) part = exact_row_dot(q, s, row, K, X + (int64_t)m * ldx, h * (K / 2), (h + 1) * (K / 2));
       part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
