@@ -70,6 +70,7 @@ struct Bars {
   uint32_t tmem_addr;
   volatile int err;
   int info[512];      // the tile's row exponents (or kWideRow), staged for the epilogue
+  float colpow[512];  // 2^-e of each row (1 for wide rows)
 };
 
 template <int BN, int NSUB>
@@ -112,6 +113,10 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Bar
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
+}
+
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
@@ -430,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = t; i < BNT; i += kDeqWarps * 32) {
       const int e = m0 + i < M ? __ldg(info + m0 + i) : 0;
       bars->info[i] = e;
+      bars->colpow[i] = e == kWideRow ? 1.0f : pow2f(-e);
       wide_here |= e == kWideRow;
     }
     const bool any_wide = group_any(1, kDeqWarps * 32, wide_here);
@@ -446,25 +452,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int c_begin = BNT >= 64 ? half_id * kColsPerWarp : 0;
       const bool active = BNT >= 64 || half_id == 0;
       if (active) {
+        // Each 32 x 32 block (weight rows n of this lane quarter, activation
+        // rows m) goes through a 2 KB staging area in the (now idle) A ring, so
+        // that Y is written as 64-byte row segments with 16-byte stores.
+        const uint32_t stage = ptx::smem_u32(a_tile(0)) + (uint32_t)(warp - kDeqWarp0) * 2048u;
+        const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
 #pragma unroll 1
         for (int c0 = c_begin; c0 < c_begin + kColsPerWarp; c0 += 32) {
           uint32_t rr[32];
           ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
           ptx::tmem_ld_wait();
-          if (n < N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int m = m0 + c0 + j;
-              if (c0 + j < c_begin + kColsPerWarp && m < M) {
-                const int e = bars->info[c0 + j];
-                if (e != kWideRow) {
-                  const float v = (__uint_as_float(rr[j]) * gv) * pow2f(-e);
-                  const __nv_bfloat16 o = __float2bfloat16_rn(v);
-                  Y[(int64_t)m * ldy + n] = *reinterpret_cast<const uint16_t*>(&o);
-                }
+          for (int j = 0; j < 32; ++j) {
+            const __nv_bfloat16 o = __float2bfloat16_rn((__uint_as_float(rr[j]) * gv) * bars->colpow[c0 + j]);
+            st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
+          }
+          __syncwarp();
+          // row j of the block: 32 consecutive n = 64 bytes, four lanes per row
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
+            const int m = m0 + c0 + j;
+            const int nb = n0 + 32 * quarter + 8 * piece;
+            if (c0 + j < c_begin + kColsPerWarp && m < M && bars->info[c0 + j] != kWideRow && nb < N) {
+              const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
+              uint16_t* dst = Y + (int64_t)m * ldy + nb;
+              if (vec_ok && nb + 8 <= N) {
+                *reinterpret_cast<uint4*>(dst) = v;
+              } else {
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
               }
             }
           }
+          __syncwarp();
         }
       }
     }
