@@ -20,8 +20,9 @@
 //   - when a stage is released, the producer warp sums the WK partials of
 //     each row in a fixed order (deterministic), applies g and 2^-e, and
 //     stores y before refilling the stage.
-// x is scanned once per CTA for its range (power-of-two scale for the exact
-// f16 operand, or the exact fp32 path), overlapped with the first copies.
+// Each compute warp scales its own K slice of x by a power of two into f16
+// (exact when the slice's range allows, else an exact fp32 path); the
+// producer undoes each slice's scale before summing the slices.
 #include "nvfp4_device.cuh"
 #include "nvfp4_kernels.h"
 #include "sm100_ptx.cuh"
@@ -156,12 +157,11 @@ __global__ void __launch_bounds__(MAXT, 1)
                        const float* __restrict__ g, uint16_t* __restrict__ y, int N, int K, StreamShape sh,
                        int static_weights) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint32_t red_max[32], red_min[32];
+  __shared__ float slice_scale[32];  // per K slice: 2^-e, e the power of two its x was scaled by
   __shared__ int s_err;
   const int wk = sh.wk, rg = sh.rg, rs = sh.rs, ns = sh.ns;
   const int n_compute = wk * rg;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
   const int row_bytes = K >> 1, row_sc = K >> 4;
   const int stage_q = rs * row_bytes, stage_bytes = rs * (row_bytes + row_sc);
   float* red = reinterpret_cast<float*>(smem + (size_t)ns * stage_bytes);
@@ -203,54 +203,54 @@ __global__ void __launch_bounds__(MAXT, 1)
     for (int i = 0; i < min(ns, nstages); ++i) issue(i, i);
   if (static_weights) asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- range of |x| over the whole vector (all warps)
-  uint32_t mx = 0, mn = 0xFFFFu;
-  for (int i = threadIdx.x; i < (K >> 3); i += blockDim.x) {
-    const uint4 v = *reinterpret_cast<const uint4*>(x + 8 * i);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
-      mx = max(mx, max(lo, hi));
-      mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
-    }
-  }
-  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-  mn = __reduce_min_sync(0xFFFFFFFFu, mn);
-  if (lane == 0) {
-    red_max[warp] = mx;
-    red_min[warp] = mn;
-  }
-  __syncthreads();
-  mx = red_max[0];
-  mn = red_min[0];
-  for (int w = 1; w < nwarps; ++w) {
-    mx = max(mx, red_max[w]);
-    mn = min(mn, red_min[w]);
-  }
-  bool fast = true;
-  int e = 0;
-  if (mx >= 0x7F80u) {
-    fast = false;
-  } else if (mx != 0) {
-    const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
-    e = 15 - hi_exp;
-    fast = hi_exp - lo_exp <= 32;
-  }
-
   if (!producer && warp < n_compute) {
     // ------------------------------------------------------------ compute
     const int kw = warp % wk, rgi = warp / wk;
     const int kbase = kw * 1024 + lane * 32;  // this lane's 32 x elements
-    uint32_t xh[16];
+    // This warp's K slice of x as f16 scaled by 2^e, e chosen from the
+    // slice's own range (exact when its non-zero magnitudes lie within 2^32
+    // of each other and it is finite; else the exact fp32 path).  The
+    // producer scales each slice's partial sums back by 2^-e before the
+    // fixed-order sum, so no block-wide pass over x is needed.
+    uint4 xv[4];
     {
       const uint4* xp = reinterpret_cast<const uint4*>(x + kbase);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) xv[c] = xp[c];
+    }
+    uint32_t mx = 0, mn = 0xFFFFu;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t w4[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
+        mx = max(mx, max(lo, hi));
+        mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
+      }
+    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+    bool fast = true;
+    int e = 0;
+    if (mx >= 0x7F80u) {
+      fast = false;
+    } else if (mx != 0) {
+      const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
+      e = 15 - hi_exp;
+      fast = hi_exp - lo_exp <= 32;
+    }
+    if (!fast) e = 0;
+    // read by the producer after the first stage: 2^-e (subnormal below 2^-126)
+    if (rgi == 0 && lane == 0)
+      slice_scale[kw] = e <= 126 ? exp2i(-e) : __uint_as_float(1u << (149 - e));
+    uint32_t xh[16];
+    {
       const int e1 = e / 2, e2 = e - e1;
       const float m1 = exp2i(e1), m2 = exp2i(e2);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const uint4 v = xp[c];
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t w4[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const __half2 h = __floats2half2_rn(bf16lo_to_float(w4[j]) * m1 * m2, bf16hi_to_float(w4[j]) * m1 * m2);
@@ -309,21 +309,24 @@ __global__ void __launch_bounds__(MAXT, 1)
     int st = 0;
     uint32_t phase = 0;
     for (int i = 0; i < nstages; ++i) {
-      if (!wait_sleep(&empty[st], phase)) {
+      // spin (no suspend): the refill below is on the critical path
+      if (!ptx::mbar_wait(&empty[st], phase, kWaitLimitNs)) {
         if (lane == 0 && atomicExch(&s_err, 1) == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
         break;
       }
+      // refill the stage first (its partial sums live in a separate buffer
+      // that is rewritten only after this refill has landed and been read)
+      if (lane == 0 && i + ns < nstages) issue(i + ns, st);
       const int rows_here = min(rs, nrows - i * rs);
       for (int r = lane; r < rows_here; r += 32) {
         const float* rp = red + (st * rs + r) * wk;
         float acc = 0.0f;
-        for (int k = 0; k < wk; ++k) acc += rp[k];
-        const float out = fast ? ldexpf(acc * gv, -e) : acc * gv;
+        for (int k = 0; k < wk; ++k) acc = fmaf(rp[k], slice_scale[k], acc);
+        const float out = acc * gv;
         const __nv_bfloat16 o = __float2bfloat16_rn(out);
         y[row_begin + i * rs + r] = *reinterpret_cast<const uint16_t*>(&o);
       }
       __syncwarp();
-      if (lane == 0 && i + ns < nstages) issue(i + ns, st);
       if (++st == ns) {
         st = 0;
         phase ^= 1u;
