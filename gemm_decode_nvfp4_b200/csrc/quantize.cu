@@ -41,10 +41,22 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
   const int64_t vpr = cols / 8;
   const int64_t total = rows * vpr;
   float m = 0.0f;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
-       t += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = t / vpr, c = (t - r * vpr) * 8;
-    m = absmax8(ld_stream_v4(w + r * ldw + c), m);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (ldw == cols) {
+    // contiguous rows: one flat array, four independent 16-byte loads in flight
+    const uint4* wv = reinterpret_cast<const uint4*>(w);
+    for (; t + 3 * stride < total; t += 4 * stride) {
+      const uint4 a = ld_stream_v4(wv + t), b = ld_stream_v4(wv + t + stride);
+      const uint4 c = ld_stream_v4(wv + t + 2 * stride), d = ld_stream_v4(wv + t + 3 * stride);
+      m = absmax8(d, absmax8(c, absmax8(b, absmax8(a, m))));
+    }
+    for (; t < total; t += stride) m = absmax8(ld_stream_v4(wv + t), m);
+  } else {
+    for (; t < total; t += stride) {
+      const int64_t r = t / vpr, c = (t - r * vpr) * 8;
+      m = absmax8(ld_stream_v4(w + r * ldw + c), m);
+    }
   }
   m = warp_max(m);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
@@ -85,6 +97,22 @@ __device__ __forceinline__ void quantize_block(const float (&f)[16], float g, ui
   codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
 }
 
+// Quantize the 16 BF16 values of (v0, v1) and store 8 code bytes and the scale.
+__device__ __forceinline__ void quantize_store(uint4 v0, uint4 v1, float g, uint8_t* qd, uint8_t* sd) {
+  const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = bf16lo_to_float(wv[i]);
+    f[2 * i + 1] = bf16hi_to_float(wv[i]);
+  }
+  uint32_t sc;
+  uint2 codes;
+  quantize_block(f, g, sc, codes);
+  *reinterpret_cast<uint2*>(qd) = codes;
+  *sd = static_cast<uint8_t>(sc);
+}
+
 __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restrict__ w, int64_t N,
                                                        int64_t K, int64_t ldw,
                                                        const float* __restrict__ amax,
@@ -95,8 +123,26 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
   if (g_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
   const int64_t bpr = K / 16;
   const int64_t total = N * bpr;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
-       t += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (ldw == K) {
+    // contiguous rows: block t reads w[16t ..], writes q[8t ..] and s[t]; two
+    // blocks (four 16-byte loads) in flight per thread
+    for (; t + stride < total; t += 2 * stride) {
+      const uint4* s0 = reinterpret_cast<const uint4*>(w + t * 16);
+      const uint4* s1 = reinterpret_cast<const uint4*>(w + (t + stride) * 16);
+      const uint4 a0 = ld_stream_v4(s0), a1 = ld_stream_v4(s0 + 1);
+      const uint4 b0 = ld_stream_v4(s1), b1 = ld_stream_v4(s1 + 1);
+      quantize_store(a0, a1, g, q + t * 8, s + t);
+      quantize_store(b0, b1, g, q + (t + stride) * 8, s + t + stride);
+    }
+    if (t < total) {
+      const uint4* s0 = reinterpret_cast<const uint4*>(w + t * 16);
+      quantize_store(ld_stream_v4(s0), ld_stream_v4(s0 + 1), g, q + t * 8, s + t);
+    }
+    return;
+  }
+  for (; t < total; t += stride) {
     const int64_t n = t / bpr, b = t - n * bpr;
     const uint16_t* src = w + n * ldw + b * 16;
     const uint4 v0 = ld_stream_v4(src), v1 = ld_stream_v4(src + 8);
