@@ -74,7 +74,7 @@ def kernel_source_hash(files) -> str:
 # counts only while these files are unchanged since the ncu capture.
 _CSRC = "gemm_decode_nvfp4_b200/csrc/"
 KERNEL_SOURCES = {
-    "gemv": [_CSRC + "gemv_stream.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
+    "gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh"],
     "quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
     "gemm_m32": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
     "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],

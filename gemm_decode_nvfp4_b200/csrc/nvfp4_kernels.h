@@ -17,15 +17,11 @@ cudaError_t launch_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw
                             const float* amax, uint8_t* q, uint8_t* s, float* g_out,
                             cudaStream_t stream, int sms);
 cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream);
-// Decode GEMV: the persistent bulk-copy kernel (gemv_stream.cu) when K is a
-// multiple of 1024 (up to 24576), else the general kernel (gemv.cu).
-// static_weights: q, s and g are not written by work still running on the
-// stream, so they may be read before it completes (programmatic dependent launch).
+// Decode GEMV (gemv.cu).  static_weights: q, s and g are not written by work
+// still running on the stream, so they may be read before it completes
+// (programmatic dependent launch).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream);
-bool gemv_stream_supported(int64_t N, int64_t K);
-cudaError_t launch_gemv_stream(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
-                               int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream);
 
 // Tensor-core GEMM (gemm_tc.cu): shapes it covers, the launcher, and the count
 // of CTAs whose bounded pipeline wait gave up since the last read.
@@ -53,7 +49,6 @@ cudaError_t launch_gemm_small(const uint16_t* X, int64_t ldx, const uint8_t* q, 
                               uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
                               bool static_weights, cudaStream_t stream);
 cudaError_t read_and_clear_small_timeouts(unsigned int* count);
-cudaError_t read_and_clear_gemv_timeouts(unsigned int* count);
 
 // Record a message for nvfp4_last_error() on this thread and return st (or
 // NVFP4_ERR_CUDA for a CUDA error), for entry points defined outside abi.cu.
