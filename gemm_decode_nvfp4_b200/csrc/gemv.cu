@@ -135,8 +135,11 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
 
   // ---- range of |x| (bit patterns of non-negative BF16 order like values)
   uint32_t mx = 0, mn = 0xFFFFu;
+  // (the raw BF16 vectors go to shared memory on the way; each thread later
+  // converts the vectors it wrote, so x is read from global memory once)
   for (int i = threadIdx.x; i < (K >> 3); i += kThreads) {
     const uint4 v = *reinterpret_cast<const uint4*>(x + 8 * i);
+    reinterpret_cast<uint4*>(xsm)[i] = v;
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
     const int e1 = e / 2, e2 = e - e1;  // two exact power-of-two steps
     const float m1 = exp2i(e1), m2 = exp2i(e2);
     for (int i = threadIdx.x; i < (K >> 3); i += kThreads) {
-      const uint4 v = *reinterpret_cast<const uint4*>(x + 8 * i);
+      const uint4 v = reinterpret_cast<const uint4*>(xsm)[i];  // written by this thread above
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
       uint32_t o[4];
 #pragma unroll
