@@ -76,7 +76,8 @@ _CSRC = "gemm_decode_nvfp4_b200/csrc/"
 KERNEL_SOURCES = {
     "gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh"],
     "quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
-    "gemm_m32": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
+    "gemm_m32": [_CSRC + "gemm_small.cu", _CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh",
+                 _CSRC + "tc_host.h"],
     "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
 }
 
