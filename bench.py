@@ -97,6 +97,25 @@ def traffic_from_profiles(row: str):
     return e.get("dram_bytes_per_call")
 
 
+# ------------------------------------------------------------ ranks (replicas)
+
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise max of per-rank timings (the replicas run independently;
+    the job ends when the slowest rank ends).  Every rank must call it."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(bytes_per_rank: float, max_ms: float, world: int) -> float:
+    """Whole-job GB/s: the bytes all ranks processed over the slowest rank's time."""
+    return bytes_per_rank * world / (max_ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------ clock sampler
 
 class ClockSampler:
@@ -290,12 +309,10 @@ def run_gpu(args):
         t = sum(a.elapsed_time(b) for a, b in evs[name])
         per_launch_ms[name] = t / (args.steps * launches)
 
-    if world > 1:
-        t = torch.tensor([total_ms] + [per_launch_ms[n] for n, *_ in rows], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t[0])
-        for i, (n, *_) in enumerate(rows):
-            per_launch_ms[n] = float(t[i + 1])
+    red = max_over_ranks([total_ms] + [per_launch_ms[n] for n, *_ in rows], world, dev)
+    total_ms = red[0]
+    for i, (n, *_) in enumerate(rows):
+        per_launch_ms[n] = red[i + 1]
 
     hbm = peaks["hbm_gbs"]
     bf16_burst = peaks["bf16_tflops"]
@@ -344,11 +361,7 @@ def run_gpu(args):
                 b.synchronize()
                 if it >= args.warmup:
                     e2e_ms.append(a.elapsed_time(b))
-    e2e_t = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_t = float(t[0])
+    e2e_t = max_over_ranks([statistics.mean(e2e_ms)], world, dev)[0]
 
     launches = 0
     for name, _, n_launch, n_kern in rows:
@@ -362,7 +375,7 @@ def run_gpu(args):
     if rank == 0:
         out = {
             "metric": METRIC,
-            "value": gemv_gbs * world,
+            "value": job_throughput(gb, per_launch_ms["gemv"], world),
             "unit": "GB/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -383,7 +396,7 @@ def run_gpu(args):
                          "peak_source": peaks["source"], "kernel": "gemv",
                          "algorithmic_bytes_per_launch": gb},
             "kernels": kernels,
-            "e2e": {"value": gb / (e2e_t * 1e-3) / 1e9 * world, "unit": "GB/s",
+            "e2e": {"value": job_throughput(gb, e2e_t, world), "unit": "GB/s",
                     "h2d_bytes_per_step": 2 * K, "d2h_bytes_per_step": 2 * N,
                     "what": "per step: pinned x H2D, nvfp4_gemv, y D2H (weights resident)"},
             "gpu_launches": launches,
