@@ -262,11 +262,13 @@ nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, con
 }
 
 nvfp4_status nvfp4_check_device_errors(void) {
-  unsigned int n = 0, k = 0;
+  unsigned int n = 0, k = 0, v = 0;
   cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_small_timeouts(&k);
+  if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_timeouts(&v);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error counter");
-  if (n || k) return fail(NVFP4_ERR_TIMEOUT, "%u GEMM and %u small-M GEMM CTA(s) gave up on a pipeline wait", n, k);
+  if (n || k || v)
+    return fail(NVFP4_ERR_TIMEOUT, "%u GEMM, %u small-M GEMM and %u GEMV CTA(s) gave up on a pipeline wait", n, k, v);
   return NVFP4_OK;
 }
 

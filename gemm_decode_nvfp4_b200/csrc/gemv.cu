@@ -16,20 +16,41 @@
 // the CTA checks while staging.  Otherwise the CTA takes the exact fp32 path
 // (x in fp32, codes -> f16 -> fp32, packed fp32x2 FMAs).  Either way every
 // product is exact and the accumulation is fp32; the result is
-// y = bf16_rn(2^-e * (g * acc)).
+// y = bf16_rn(2^-e * (g * acc)).  The weight stream (0.5625 B/weight) is the
+// roofline: HBM bandwidth.
 //
-// Work split: a warp owns R = 8 consecutive rows; lane l reads the 16-byte
-// chunks l, l+32, ... of each row (512 contiguous bytes per warp-load, one
-// 16-bit scale load per chunk).  Two register buffers alternate (the step
-// loop is unrolled by two, so no buffer is copied): the next step's 8 x 16
-// bytes per lane are in flight while the current step is computed.  Launched
-// with programmatic dependent launch; with static weights the first loads are
-// issued before the previous kernel has finished.  The weight stream (0.5625
-// B/weight) is the roofline: HBM bandwidth.
+// Two kernels:
+//
+// * Ring kernel (K a multiple of 256, K <= 11520): one CTA per SM holding half
+//   of the SM's registers and shared memory, so that the next kernel on the
+//   stream can be resident beside it.  CTA c owns a contiguous range of about
+//   N / #SMs rows.  A producer thread streams the range through a ring of
+//   shared-memory stages with 2-D TMA copies (120 rows x 256 code bytes + their
+//   scales per stage; rows past the end read as zero); 15 consumer warps own
+//   4 rows x one 16-byte chunk per lane, release a stage as soon as its bytes
+//   are in registers, and reduce each row over its 16 lanes once.  After the
+//   previous kernel has finished, x arrives first (one bulk copy), then the
+//   ring, so x is never queued behind weight traffic.  The next kernel on the
+//   stream may start (programmatic dependent launch) once this one has staged
+//   x; its CTAs then wait in the other half of each SM.  The static-weights
+//   flag does not change this kernel: weight requests issued before x, by it
+//   or by the kernel after it, were measured to delay x more than they saved.
+//
+// * Register kernel (every other K): a warp owns R = 8 consecutive rows; lane l
+//   reads the 16-byte chunks l, l+32, ... of each row into two register buffers
+//   that alternate, the next step's loads in flight while the current step is
+//   computed.
 #include "nvfp4_kernels.h"
 #include "nvfp4_device.cuh"
+#include "sm100_ptx.cuh"
+#include "tc_host.h"
+
+#include <algorithm>
 
 namespace nvfp4 {
+
+// CTAs of the ring kernel whose bounded pipeline wait gave up since the last read.
+__device__ unsigned int g_gemv_wait_timeouts = 0;
 
 namespace {
 
@@ -288,13 +309,323 @@ cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const 
   return cudaLaunchKernelEx(&cfg, kern, x, q, s, g, y, N, K, static_weights ? 1 : 0);
 }
 
+
+// ------------------------------------------------------------------------------------------ ring kernel
+
+constexpr int kRingConsumerWarps = 15;                    // warp 15 is the producer
+constexpr int kRingConsumers = kRingConsumerWarps * 32;   // 480 threads
+constexpr int kRingThreads = kRingConsumers + 32;         // 512 threads x 64 registers: half an SM
+constexpr int kRingBK = 256;                              // code bytes of a row per stage (512 weights)
+constexpr int kRingChunks = kRingBK / 16;                 // 16 lanes share a row
+constexpr int kRingRows = 4;                              // rows per lane
+constexpr int kRingMaxBR = (kRingConsumers / kRingChunks) * kRingRows;  // 120 rows per stage
+constexpr int kRingScOff = kRingMaxBR * kRingBK;          // scales start after a fixed 120-row code block
+constexpr int kRingStage = kRingScOff + kRingMaxBR * (kRingBK / 8);   // 34560 bytes
+constexpr int kRingMaxK = kRingConsumers * 24;            // x: at most 3 uint4 per consumer thread
+constexpr uint64_t kRingWaitNs = 2000000000ull;
+
+__device__ __forceinline__ void ring_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
+
+__device__ __forceinline__ void tma_load_2d_evict_first(void* dst, const void* tmap, uint64_t* bar, int c0, int c1,
+                                                        uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(ptx::smem_u32(dst)),
+      "l"(tmap), "r"(ptx::smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+
+// Shared memory: S stages of kRingStage bytes, then x (nks x 1 KB: f16, each
+// stage's 512 values laid out [word i][chunk c] so that a quarter-warp reads
+// 128 contiguous bytes), then the barriers and the reduction scratch.
+// Rows of a CTA: [blockIdx.x * nblk * BR, + nblk * BR), in nblk blocks of BR
+// rows (BR <= 120) that go through the ring one 256-byte column at a time.
+__global__ void __launch_bounds__(kRingThreads, 2)
+    gemv_ring_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
+                     const uint16_t* __restrict__ x, const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
+                     const float* __restrict__ g, uint16_t* __restrict__ y, int N, int K, int BR, int nblk,
+                     int S) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  const int nks = (K / 2 + kRingBK - 1) / kRingBK;  // stages per row block
+  uint8_t* ring = sm;
+  uint4* xs = reinterpret_cast<uint4*>(sm + S * kRingStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xs + nks * 64);
+  uint64_t* empty = full + S;
+  uint64_t* xfull = empty + S;
+  uint32_t* red = reinterpret_cast<uint32_t*>(xfull + 1);        // [2][16]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 32);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row_base = blockIdx.x * nblk * BR;
+  const int nb_here = min(nblk, (N - row_base + BR - 1) / BR);
+  const int total = nb_here * nks;
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kRingConsumerWarps);
+    }
+    ptx::mbar_init(xfull, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kRingConsumerWarps) {  // ------------------------------------------------- producer
+    if (lane != 0) return;
+    ptx::prefetch_tmap(&tq);
+    ptx::prefetch_tmap(&ts);
+    uint64_t policy;  // each weight byte is read once: do not keep it in L2
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+    int n = 0, slot = 0, t = 0, rb = 0;
+    uint32_t phase = 0;
+    auto issue = [&]() {
+      uint8_t* dst = ring + slot * kRingStage;
+      const int row0 = row_base + rb * BR;
+      ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)BR * (kRingBK + kRingBK / 8));
+      tma_load_2d_evict_first(dst, &tq, &full[slot], t * kRingBK, row0, policy);
+      tma_load_2d_evict_first(dst + kRingScOff, &ts, &full[slot], t * (kRingBK / 8), row0, policy);
+      if (++slot == S) { slot = 0; phase ^= 1; }
+      if (++t == nks) { t = 0; ++rb; }
+    };
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x and the weights only after this
+    ptx::mbar_arrive_expect_tx(xfull, (uint32_t)K * 2);
+    ptx::bulk_load(xs, x, (uint32_t)K * 2, xfull);
+    for (; n < total; ++n) {
+      if (n >= S) {  // wait until the consumers have released this slot (or have given up on the ring)
+        bool ok = ptx::mbar_try_wait(&empty[slot], phase ^ 1);
+        const uint64_t t0 = ok ? 0 : ptx::globaltimer_ns();
+        while (!ok && !*abort_flag) {
+          if (ptx::globaltimer_ns() - t0 > kRingWaitNs) {
+            atomicAdd(&g_gemv_wait_timeouts, 1u);
+            break;
+          }
+          ok = ptx::mbar_try_wait(&empty[slot], phase ^ 1);
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) break;
+      issue();
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // nothing may still be landing in shared memory when the CTA exits
+    for (int m = max(0, n - S); m < n; ++m) ptx::mbar_wait(&full[m % S], (m / S) & 1, kRingWaitNs);
+    ptx::mbar_wait(xfull, 0, kRingWaitNs);
+    return;
+  }
+
+  // ------------------------------------------------------------------------------- consumers
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // y is written only after the previous kernel
+  if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(xfull, 0, kRingWaitNs))) {
+    if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+    *abort_flag = 1;
+    return;
+  }
+  // range of |x| over the raw BF16 bit patterns, which stay in registers
+  const int nx = K >> 3;
+  uint4 raw[3];
+  uint32_t mx = 0, mn = 0xFFFFu;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int u = tid + k * kRingConsumers;
+    raw[k] = u < nx ? xs[u] : make_uint4(0, 0, 0, 0);
+    const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
+      mx = max(mx, max(lo, hi));
+      mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
+    }
+  }
+  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+  mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+  if (lane == 0) { red[warp] = mx; red[16 + warp] = mn; }
+  ring_sync(kRingConsumers);  // every raw value is in registers: the buffer may be overwritten
+  mx = red[0]; mn = red[16];
+#pragma unroll
+  for (int w = 1; w < kRingConsumerWarps; ++w) { mx = max(mx, red[w]); mn = min(mn, red[16 + w]); }
+  bool fast = true;
+  int e = 0;
+  if (mx >= 0x7F80u) {
+    fast = false;
+  } else if (mx != 0) {
+    const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
+    e = 15 - hi_exp;
+    fast = hi_exp - lo_exp <= 32;
+  }
+  const float gv = *g;
+  if (!fast) {  // x outside the f16 window: the producer stops, every warp takes rows exactly
+    *abort_flag = 1;
+    const int nrows = min(N - row_base, nblk * BR);
+    for (int r = warp; r < nrows; r += kRingConsumerWarps) gemv_rows_exact(x, q, s, gv, y, N, K, row_base + r, 1);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
+  {
+    const int e1 = e / 2, e2 = e - e1;  // two exact power-of-two steps
+    const float m1 = exp2i(e1), m2 = exp2i(e2);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int u = tid + k * kRingConsumers;  // x[8u .. 8u+8): stage u/64, chunk (u%64)/4, word u%4
+      if (u < nx) {
+        const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = __floats2half2_rn(bf16lo_to_float(w4[j]) * m1 * m2, bf16hi_to_float(w4[j]) * m1 * m2);
+          o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    // the last stage's columns past K meet zero codes: their x must be finite
+    for (int u = nx + tid; u < nks * 64; u += kRingConsumers)
+      xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(0, 0, 0, 0);
+  }
+  ring_sync(kRingConsumers);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may now take the other half
+
+  // lane: rows r0 .. r0+3 of the 120-row stage layout, 16-byte chunk c of each
+  // (rows at or past BR hold stale bytes; their sums are never stored)
+  const int c = tid & (kRingChunks - 1);
+  const int r0 = (tid / kRingChunks) * kRingRows;
+  const uint8_t* lane_codes = ring + r0 * kRingBK + c * 16;
+  const uint8_t* lane_scales = ring + kRingScOff + r0 * (kRingBK / 8) + 2 * c;
+  const uint4* lane_x = xs + c;
+  int slot = 0;
+  uint32_t phase = 0;
+  for (int rb = 0; rb < nb_here; ++rb) {
+    float acc[kRingRows] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int t = 0; t < nks; ++t) {
+      if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&full[slot], phase, kRingWaitNs))) {
+        if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+        *abort_flag = 1;
+        return;
+      }
+      const uint8_t* pc = lane_codes + slot * kRingStage;
+      const uint8_t* ps = lane_scales + slot * kRingStage;
+      uint4 cw[kRingRows];
+      uint32_t sc[kRingRows];
+#pragma unroll
+      for (int i = 0; i < kRingRows; ++i) {
+        cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingBK);
+        sc[i] = *reinterpret_cast<const uint16_t*>(ps + i * (kRingBK / 8));
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[slot]);  // the stage's bytes are in registers
+      if (++slot == S) { slot = 0; phase ^= 1; }
+      const uint4* xp = lane_x + t * 64;
+      float part[kRingRows][2];
+#pragma unroll
+      for (int i = 0; i < kRingRows; ++i) part[i][0] = part[i][1] = 0.0f;
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {  // 8 weights per 32-bit word; words 0-1 block 0, words 2-3 block 1
+        const uint4 xv = xp[wi * 16];
+#pragma unroll
+        for (int i = 0; i < kRingRows; ++i) {
+          const uint32_t word = wi == 0 ? cw[i].x : wi == 1 ? cw[i].y : wi == 2 ? cw[i].z : cw[i].w;
+          float p = part[i][wi >> 1];
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
+          part[i][wi >> 1] = p;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kRingRows; ++i) {
+        const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
+        acc[i] = fmaf(part[i][0], sf.x, acc[i]);
+        acc[i] = fmaf(part[i][1], sf.y, acc[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kRingRows; ++i) {
+      float v = acc[i];
+#pragma unroll
+      for (int o = kRingChunks / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+      acc[i] = v;
+    }
+    if (c < kRingRows) {
+      const float v = c == 0 ? acc[0] : c == 1 ? acc[1] : c == 2 ? acc[2] : acc[3];
+      const int rl = r0 + c;
+      const int row = row_base + rb * BR + rl;
+      if (rl < BR && row < N) {
+        const __nv_bfloat16 o = __float2bfloat16_rn(ldexpf(v * gv, -e));
+        y[row] = *reinterpret_cast<const uint16_t*>(&o);
+      }
+    }
+  }
+}
+
+struct RingPlan {
+  int BR, nblk, grid, S;
+  size_t smem;
+};
+
+// The ring kernel's shape: rows split evenly over the SMs, shared memory for at
+// least two stages within half of the SM.  False when K does not fit it.
+bool ring_plan(int64_t N, int64_t K, int sms, RingPlan& p) {
+  if (K % 256 != 0 || K > kRingMaxK || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
+  int dev = 0, per_sm = 0, reserved = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return false;
+  const int64_t rpc = (N + sms - 1) / sms;
+  p.nblk = (int)((rpc + kRingMaxBR - 1) / kRingMaxBR);
+  p.BR = (int)((rpc + p.nblk - 1) / p.nblk);
+  p.grid = (int)((N + (int64_t)p.nblk * p.BR - 1) / ((int64_t)p.nblk * p.BR));
+  const int64_t nks = (K / 2 + kRingBK - 1) / kRingBK;
+  const int64_t fixed = nks * 1024 + 256;
+  const int64_t budget = per_sm / 2 - reserved;  // two such CTAs per SM
+  if (fixed + 2 * kRingStage > budget) return false;
+  p.S = (int)std::min<int64_t>(4, (budget - fixed) / kRingStage);
+  p.smem = (size_t)(p.S * kRingStage + fixed);
+  return true;
+}
+
+cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
+                        int64_t N, int64_t K, cudaStream_t stream, const RingPlan& p, bool* encoded) {
+  CUtensorMap tq, ts;
+  *encoded = tc::make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, N, K / 2, kRingBK, p.BR,
+                              CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             tc::make_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, K / 16, N, K / 16, kRingBK / 8, p.BR,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!*encoded) return cudaSuccess;
+  static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || smem_set[dev] < (int)p.smem) {
+    e = cudaFuncSetAttribute(gemv_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) smem_set[dev] = (int)p.smem;
+  }
+  int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S;
+  void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S};
+  return tc::launch_pdl((const void*)gemv_ring_kernel, dim3(p.grid), dim3(kRingThreads), p.smem, stream, args);
+}
+
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  (void)sms;
+  RingPlan plan;
+  if (ring_plan(N, K, sms, plan)) {
+    bool encoded = false;
+    const cudaError_t e = launch_ring(x, q, s, g, y, N, K, stream, plan, &encoded);
+    if (encoded || e != cudaSuccess) return e;
+  }
   if (K % 32 == 0) return launch<8, 16, 2>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
   return launch<8, 8, 2>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
+}
+
+cudaError_t read_and_clear_gemv_timeouts(unsigned int* count) {
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_gemv_wait_timeouts, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_gemv_wait_timeouts, &zero, sizeof(unsigned int));
 }
 
 }  // namespace nvfp4

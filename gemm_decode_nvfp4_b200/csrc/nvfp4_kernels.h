@@ -22,6 +22,8 @@ cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream);
 // (programmatic dependent launch).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream);
+// CTAs of the decode GEMV whose bounded pipeline wait gave up since the last read.
+cudaError_t read_and_clear_gemv_timeouts(unsigned int* count);
 
 // Tensor-core GEMM (gemm_tc.cu): shapes it covers, the launcher, and the count
 // of CTAs whose bounded pipeline wait gave up since the last read.

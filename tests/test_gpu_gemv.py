@@ -218,3 +218,28 @@ def test_quantize_then_gemv_same_stream(nv):
     q_ref, s_ref, g_ref = oracle.quantize(w.cpu())
     y_ref, bound = oracle.linear(x.cpu().reshape(1, -1), q_ref, s_ref, g_ref)
     assert_within_tolerance(y, y_ref[0], bound[0], "quantize->gemv")
+
+
+@pytest.mark.parametrize("N,K", [(148 * 120 + 7, 2048),   # two row blocks per CTA
+                                 (148 * 118 + 1, 1024),   # short last CTA
+                                 (333, 1280),             # last 256-byte column half past K
+                                 (3, 768), (1, 256),
+                                 (500, 11520),            # largest K of the shared-memory ring
+                                 (64, 11776)])            # next multiple of 256: register kernel
+@pytest.mark.parametrize("static", [False, True])
+def test_ring_shapes(nv, N, K, static):
+    """Shapes at the edges of the TMA-ring GEMV (K a multiple of 256): rows
+    split over the SMs in one or more blocks, ragged last blocks and columns,
+    both weight-ordering flags; the device error counter stays clear."""
+    q, s = workloads.random_codes(N, K, 3 * N + K)
+    x = workloads.random_bf16((1, K), N + 5 * K)
+    g = np.float32(0.011)
+    y_ref, bound = oracle.linear(x, q.numpy(), s.numpy(), g)
+    xd = x.reshape(-1).cuda()
+    qd, sd = q.cuda(), s.cuda()
+    gd = torch.tensor([float(g)], dtype=torch.float32, device="cuda")
+    y, check = guarded_empty((N,), torch.bfloat16)
+    nv.gemv(xd, qd, sd, gd, y, static_weights=static)
+    check()
+    assert_within_tolerance(y, y_ref[0], bound[0], f"N={N} K={K} static={static}")
+    nv.check_device_errors()
