@@ -206,8 +206,8 @@ NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint16_t* X, int64_t ldx, const 
                                           int64_t K, uint32_t flags, nvfp4_stream_t stream);
 
 /*
- * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMMs)
- * is bounded (about 2 s); a CTA that gives up
+ * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMMs
+ * and the TMA-fed decode GEMV) is bounded (about 2 s); a CTA that gives up
  * records it in a device counter and finishes without hanging, leaving its
  * outputs undefined.  This call reads and
  * clears that counter for the current device (it waits for prior work on the
