@@ -61,6 +61,15 @@ def lib():
         L.oracle_linear.argtypes = [c_p, c_i64, c_p, c_p, c_f, c_i64, c_i64, c_i64,
                                     c_p, c_p, c_i64, c_p, c_p]
         L.oracle_linear.restype = None
+        L.oracle_e8m0_decode.argtypes = [ctypes.c_int]
+        L.oracle_e8m0_decode.restype = ctypes.c_double
+        L.oracle_mx_quantize.argtypes = [c_p, c_i64, c_i64, c_i64, c_p, c_p]
+        L.oracle_mx_quantize.restype = None
+        L.oracle_mx_dequantize.argtypes = [c_p, c_p, c_i64, c_i64, c_p]
+        L.oracle_mx_dequantize.restype = None
+        L.oracle_mx_linear.argtypes = [c_p, c_i64, c_p, c_p, c_i64, c_i64, c_i64,
+                                       c_p, c_p, c_i64, c_p, c_p]
+        L.oracle_mx_linear.restype = None
         L.oracle_num_threads.argtypes = []
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
@@ -178,3 +187,57 @@ def linear(x, q: np.ndarray, s: np.ndarray, g, rows=None, cols=None):
 def tolerance(y_ref: np.ndarray, bound: np.ndarray) -> np.ndarray:
     """Acceptance bound per output: 1e-3 * sum|w x| + 1e-2 * |y_ref|."""
     return 1e-3 * bound + 1e-2 * np.abs(y_ref)
+
+
+# ------------------------------------------------------------------ MXFP4
+
+def e8m0_decode(byte: int) -> float:
+    return lib().oracle_e8m0_decode(int(byte))
+
+
+def mx_quantize(w):
+    """Round-to-nearest MXFP4 of a BF16 [N, K] matrix (K % 32 == 0).
+    Returns (q [N, K/2] u8, s [N, K/32] u8 UE8M0)."""
+    b = _bf16_bits(w)
+    N, K = b.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    q = np.empty((N, K // 2), np.uint8)
+    s = np.empty((N, K // 32), np.uint8)
+    lib().oracle_mx_quantize(_ptr(b), N, K, K, _ptr(q), _ptr(s))
+    return q, s
+
+
+def mx_dequantize(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """W_deq [N, K] in fp64."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    N, K = q.shape[0], q.shape[1] * 2
+    out = np.empty((N, K), np.float64)
+    lib().oracle_mx_dequantize(_ptr(q), _ptr(s), N, K, _ptr(out))
+    return out
+
+
+def mx_linear(x, q: np.ndarray, s: np.ndarray, rows=None, cols=None):
+    """MXFP4 y = x . W^T in fp64 with the bound sum |w x| (as ``linear``)."""
+    xb = _bf16_bits(x)
+    if xb.ndim == 1:
+        xb = xb.reshape(1, -1)
+    M, K = xb.shape
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    N = q.shape[0]
+    assert q.shape[1] * 2 == K and s.shape == (N, K // 32)
+    if rows is None:
+        y = np.empty((M, N), np.float64)
+        bound = np.empty((M, N), np.float64)
+        lib().oracle_mx_linear(_ptr(xb), K, _ptr(q), _ptr(s), M, N, K, None, None, -1, _ptr(y), _ptr(bound))
+        return y, bound
+    ri = np.ascontiguousarray(rows, np.int64)
+    ci = np.ascontiguousarray(cols, np.int64)
+    assert ri.shape == ci.shape and ri.ndim == 1
+    y = np.empty(ri.shape, np.float64)
+    bound = np.empty(ri.shape, np.float64)
+    lib().oracle_mx_linear(_ptr(xb), K, _ptr(q), _ptr(s), M, N, K, _ptr(ri), _ptr(ci), len(ri),
+                           _ptr(y), _ptr(bound))
+    return y, bound

@@ -44,6 +44,21 @@
  *       d = decode(s) * g;  r = 1 / d;  code = E2M1(w * r) saturating at 6,
  *       ties to the even code, sign kept.  g == 0 gives s = 0; d == 0 gives
  *       sixteen 0x0 codes; an input of +-0 gives code 0x0 / 0x8.
+ *
+ * MXFP4 ([p3] imp docs/quantization.md, the MXFP4 paragraph after the NVFP4
+ * pipelines, and the MXFP4 row of the format table): the same E2M1 nibble
+ * layout as NVFP4, one UE8M0 micro-scale per 32 elements, no tensor scale;
+ * its quantizer is round-to-nearest.  The pages give no scale formula:
+ *   R6  UE8M0 is an unsigned power of two: byte b means 2^(b - 127) for
+ *       b = 0..254; 255 is NaN.
+ *   R7  block scale X = 2^(floor(log2(amax_b)) - 2): 2 is the largest E2M1
+ *       exponent (6 = 1.5 * 2^2), so the block's largest magnitude lands in
+ *       [4, 8) before rounding.  The byte is clamped to 0..254; a block whose
+ *       elements are all zero gets byte 0.
+ *   R8  element codes: E2M1 round to nearest even of w / X (an exact
+ *       division by a power of two, done in fp64), saturating at 6, sign kept
+ *       (R5's rule).
+ *   R9  packing as R3, with scale j covering elements 32j .. 32j+31.
  */
 #include <math.h>
 #include <stdint.h>
@@ -117,10 +132,10 @@ int oracle_e4m3_rne_satfinite(float v) {
   return (sign << 7) | code;
 }
 
-/* E2M1 round-to-nearest-even with saturation to +-6, sign kept (R5). */
-int oracle_e2m1_rne_satfinite(float v) {
+/* E2M1 round-to-nearest-even with saturation to +-6, sign kept (R5, R8). */
+static int e2m1_rne_satfinite_d(double v) {
   int sign = signbit(v) ? 1 : 0;
-  double a = fabs((double)v);
+  double a = fabs(v);
   int best = 0;
   if (a > 6.0) {
     best = 7;
@@ -132,6 +147,8 @@ int oracle_e2m1_rne_satfinite(float v) {
   }
   return (sign << 3) | best;
 }
+
+int oracle_e2m1_rne_satfinite(float v) { return e2m1_rne_satfinite_d((double)v); }
 
 /* ---------------------------------------------------------- tensor scale */
 
@@ -238,6 +255,92 @@ void oracle_linear(const uint16_t* x, int64_t ldx, const uint8_t* q,
     }
     y[t] = (double)g * acc;
     bound[t] = fabs((double)g) * mag;
+  }
+}
+
+/* ------------------------------------------------------------------ MXFP4 */
+
+/* R6: UE8M0 byte -> 2^(b - 127); 255 is NaN. */
+double oracle_e8m0_decode(int byte) {
+  byte &= 255;
+  return byte == 255 ? NAN : ldexp(1.0, byte - 127);
+}
+
+/* [p3] round-to-nearest MXFP4 of a BF16 [N, K] matrix (K a multiple of 32):
+ * q [N, K/2] as R3, s [N, K/32] UE8M0 bytes (R7), codes by R8. */
+void oracle_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                        uint8_t* q, uint8_t* s) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t b = 0; b < K / 32; ++b) {
+      const uint16_t* blk = w + n * ldw + b * 32;
+      double amax_b = 0.0;
+      int codes[32];
+      for (int i = 0; i < 32; ++i) {
+        double a = fabs(oracle_bf16_to_double(blk[i]));
+        if (a > amax_b) amax_b = a;
+      }
+      int byte = 0;
+      if (amax_b > 0.0) {
+        int e2;                       /* amax_b = m * 2^e2 with m in [0.5, 1) */
+        frexp(amax_b, &e2);
+        int e = (e2 - 1) - 2;         /* floor(log2(amax_b)) - 2 */
+        byte = e + 127;
+        if (byte < 0) byte = 0;
+        if (byte > 254) byte = 254;
+      }
+      double x_scale = oracle_e8m0_decode(byte);
+      for (int i = 0; i < 32; ++i) {
+        double wi = oracle_bf16_to_double(blk[i]);
+        codes[i] = e2m1_rne_satfinite_d(wi / x_scale);
+      }
+      s[n * (K / 32) + b] = (uint8_t)byte;
+      for (int i = 0; i < 32; i += 2)
+        q[n * (K / 2) + b * 16 + i / 2] = (uint8_t)(codes[i] | (codes[i + 1] << 4));
+    }
+  }
+}
+
+/* W_deq[n, k] = e8m0(s[n, k/32]) * e2m1(q[n, k]) in fp64. */
+void oracle_mx_dequantize(const uint8_t* q, const uint8_t* s, int64_t N, int64_t K, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) {
+      uint8_t byte = q[n * (K / 2) + k / 2];
+      int code = (k % 2 == 0) ? (byte & 15) : (byte >> 4);
+      out[n * K + k] = oracle_e8m0_decode(s[n * (K / 32) + k / 32]) * oracle_e2m1_decode(code);
+    }
+}
+
+/* MXFP4 weight-only linear, y = x . W^T, outputs selected as in
+ * oracle_linear:
+ *   y[m, n]    = sum_b e8m0(s[n, b]) * sum_i e2m1(q[n, 32b+i]) * x[m, 32b+i]
+ *   bound[m,n] = sum_k |W_deq[n, k] * x[m, k]|      (fp64) */
+void oracle_mx_linear(const uint16_t* x, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                      int64_t M, int64_t N, int64_t K, const int64_t* m_idx, const int64_t* n_idx,
+                      int64_t count, double* y, double* bound) {
+  int64_t total = count < 0 ? M * N : count;
+#pragma omp parallel for schedule(dynamic, 64)
+  for (int64_t t = 0; t < total; ++t) {
+    int64_t m = count < 0 ? t / N : m_idx[t];
+    int64_t n = count < 0 ? t % N : n_idx[t];
+    double acc = 0.0, mag = 0.0;
+    for (int64_t b = 0; b < K / 32; ++b) {
+      double sb = oracle_e8m0_decode(s[n * (K / 32) + b]);
+      double part = 0.0, part_mag = 0.0;
+      for (int i = 0; i < 32; ++i) {
+        int64_t k = b * 32 + i;
+        uint8_t byte = q[n * (K / 2) + k / 2];
+        int code = (k % 2 == 0) ? (byte & 15) : (byte >> 4);
+        double prod = oracle_e2m1_decode(code) * oracle_bf16_to_double(x[m * ldx + k]);
+        part += prod;
+        part_mag += fabs(prod);
+      }
+      acc += sb * part;
+      mag += sb * part_mag;
+    }
+    y[t] = acc;
+    bound[t] = mag;
   }
 }
 
