@@ -51,6 +51,16 @@ def quantize_bytes(N: int, K: int) -> int:
     return 2 * (2 * N * K) + N * K // 2 + N * K // 16
 
 
+def mx_gemv_bytes(N: int, K: int) -> int:
+    """MXFP4 decode GEMV: nibbles + one UE8M0 byte per 32 + x + y (no tensor scale)."""
+    return N * K // 2 + N * K // 32 + 2 * K + 2 * N
+
+
+def mx_quantize_bytes(N: int, K: int) -> int:
+    """One pass: read W, write q and s (the scales need no tensor amax)."""
+    return 2 * N * K + N * K // 2 + N * K // 32
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -79,6 +89,8 @@ KERNEL_SOURCES = {
     "gemm_m32": [_CSRC + "gemm_small.cu", _CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh",
                  _CSRC + "tc_host.h"],
     "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
+    "mx_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
 }
 
 
@@ -240,12 +252,27 @@ def run_gpu(args):
         for i in range(copies):
             nv.gemv(x1, qs[i], ss[i], g0, y1[i])
 
+    # MXFP4 (UE8M0 scale per 32, no tensor scale) of the same layer, 8 copies
+    mq0, ms0 = nv.mx_quantize_new(workloads.weight_bf16(workloads.CONFIGS["decode"]).to(dev))
+    mqs = [mq0] + [mq0.clone() for _ in range(copies - 1)]
+    mss = [ms0] + [ms0.clone() for _ in range(copies - 1)]
+    mq_out = torch.empty_like(mq0)
+    ms_out = torch.empty_like(ms0)
+
+    def mx_gemv_all():
+        for i in range(copies):
+            nv.mx_gemv(x1, mqs[i], mss[i], y1[i], static_weights=True)
+
+    def mx_quant_all():
+        nv.mx_quantize(wq_in, mq_out, ms_out)
+
     def quant_all():
         amax_buf.zero_()
         nv.amax(wq_in, amax_buf)
         nv.quantize(wq_in, qq, sq, gq, amax=amax_buf)
 
     rows.append(("quantize", quant_all, 1, 2))
+    rows.append(("mx_quantize", mx_quant_all, 1, 1))
     if gemm_ok:
         def m32_all():
             for i in range(copies):
@@ -257,6 +284,7 @@ def run_gpu(args):
 
         rows.append(("gemm_m512", m512_all, copies, 2))
         rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
+    rows.append(("mx_gemv", mx_gemv_all, copies, 1))
     rows.append(("gemv_ordered", gemv_ordered_all, copies, 1))
     rows.append(("gemv", gemv_all, copies, 1))
     if args.only != "all":  # profiling runs: keep only the named row (plus the headline GEMV)
@@ -331,6 +359,17 @@ def run_gpu(args):
         qgbs = qb / (per_launch_ms["quantize"] * 1e-3) / 1e9
         kernels["quantize"] = {"us": per_launch_ms["quantize"] * 1e3, "GB/s": qgbs, "frac_hbm": qgbs / hbm,
                                "bytes": qb}
+    if "mx_gemv" in per_launch_ms:
+        mb = mx_gemv_bytes(N, K)
+        mg = mb / (per_launch_ms["mx_gemv"] * 1e-3) / 1e9
+        kernels["mx_gemv"] = {"us": per_launch_ms["mx_gemv"] * 1e3, "GB/s": mg, "frac_hbm": mg / hbm, "bytes": mb,
+                              "weight_bytes_per_token": N * K // 2 + N * K // 32,
+                              "format": "MXFP4: UE8M0 scale per 32, no tensor scale"}
+    if "mx_quantize" in per_launch_ms:
+        mb = mx_quantize_bytes(N, K)
+        mq = mb / (per_launch_ms["mx_quantize"] * 1e-3) / 1e9
+        kernels["mx_quantize"] = {"us": per_launch_ms["mx_quantize"] * 1e3, "GB/s": mq, "frac_hbm": mq / hbm,
+                                  "bytes": mb}
     for name, M in (("gemm_m32", 32), ("gemm_m512", 512)):
         if name in per_launch_ms:
             t = per_launch_ms[name] * 1e-3
@@ -389,9 +428,9 @@ def run_gpu(args):
             "config": {"workload": WORKLOAD, "N": N, "K": K, "M": 1, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {copies} rotating weight copies "
                              f"({copies * (N * K // 2 + N * K // 16) / 1e6:.0f} MB) per graph",
-                       "row_order": "quantize, gemm M=512, gemm M=32, gemv ordered, gemv static: each GEMV graph "
+                       "row_order": "quantize, MXFP4 quantize, gemm M=512, gemm M=32, MXFP4 gemv, gemv ordered, gemv static: each GEMV graph "
                                     "follows GEMVs, not the rows that leave tens of MB of dirty output in L2",
-                       "step": "quantize [17408,5120] + gemm M=512 + gemm M=32 + gemv M=1 (x2: ordered and static-weights)",
+                       "step": "quantize [17408,5120] (NVFP4, MXFP4) + gemm M=512 + gemm M=32 + MXFP4 gemv + gemv M=1 (x2: ordered and static-weights)",
             "gemv_launch": "8 GEMVs per graph on 8 weight copies, programmatic dependent launch (static weights)"},
             "roofline": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemv_gbs / hbm, "traffic": traffic,
@@ -486,7 +525,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=17408)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "gemm_m32",
-                                                      "gemm_m512"],
+                                                      "gemm_m512", "mx_gemv", "mx_quantize"],
                     help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps

@@ -22,11 +22,13 @@ __all__ = [
     "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
     "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
+    "mx_quantize", "mx_quantize_new", "mx_gemv",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
+MX_HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "mxfp4.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python gemm_decode_nvfp4_b200/build.py`")
@@ -45,10 +47,14 @@ lib.nvfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _
 lib.nvfp4_gemm_ex.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_noalloc.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
+lib.mxfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p]
+lib.mxfp4_gemv.argtypes = [_p, _p, _p, _p, _i64, _i64, _p]
+lib.mxfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
 for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
-           lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors):
+           lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors, lib.mxfp4_quantize, lib.mxfp4_gemv,
+           lib.mxfp4_gemv_ex):
     _f.restype = ctypes.c_int
 
 
@@ -75,10 +81,12 @@ def version() -> int:
 
 
 def declared_symbols() -> list[str]:
-    """Names of the entry points include/nvfp4.h declares."""
-    with open(HEADER_PATH) as f:
-        text = f.read()
-    return re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(nvfp4_\w+)\s*\(", text)
+    """Names of the entry points include/nvfp4.h and include/mxfp4.h declare."""
+    names = []
+    for path in (HEADER_PATH, MX_HEADER_PATH):
+        with open(path) as f:
+            names += re.findall(r"NVFP4_API\s+[\w\s\*]+?\b((?:nvfp4|mxfp4)_\w+)\s*\(", f.read())
+    return names
 
 
 def _stream(stream=None) -> int:
@@ -234,3 +242,45 @@ def linear(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, s
     ws = torch.empty((n_ws,), dtype=torch.uint8, device=X.device) if n_ws else None
     gemm(X2, q, s, g, Y, workspace=ws, stream=stream)
     return Y if X.dim() == 2 else Y.reshape(-1)
+
+
+# ---------------------------------------------------------------------- MXFP4
+# imp docs/quantization.md, MXFP4 paragraph: NVFP4's nibble layout with one UE8M0
+# micro-scale per 32 elements and no tensor scale (include/mxfp4.h).
+
+def mx_quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, stream=None) -> None:
+    """Round-to-nearest MXFP4 of BF16 w [N, K] into q [N, K/2] and s [N, K/32]."""
+    _need(w, torch.bfloat16, "w", 2)
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    N, K = w.shape
+    if w.stride(1) != 1 or not q.is_contiguous() or not s.is_contiguous():
+        raise ValueError("w rows and q, s must be contiguous")
+    if q.shape != (N, K // 2) or s.shape != (N, K // 32):
+        raise ValueError("q/s must be [N, K/2] / [N, K/32]")
+    _check("mxfp4_quantize", lib.mxfp4_quantize(_ptr(w), N, K, w.stride(0), _ptr(q), _ptr(s), _stream(stream)))
+
+
+def mx_quantize_new(w: torch.Tensor, stream=None):
+    """Allocate q, s on w's device and MXFP4-quantize into them."""
+    N, K = w.shape
+    q = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    s = torch.empty((N, K // 32), dtype=torch.uint8, device=w.device)
+    mx_quantize(w, q, s, stream=stream)
+    return q, s
+
+
+def mx_gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, y: torch.Tensor, stream=None,
+            static_weights: bool = False) -> None:
+    """y[N] = bf16(W_deq . x) for MXFP4 weights and BF16 x [K]."""
+    _need(x, torch.bfloat16, "x")
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    _need(y, torch.bfloat16, "y")
+    N, K = q.shape[0], q.shape[1] * 2
+    if x.numel() != K or y.numel() != N or not x.is_contiguous() or not y.is_contiguous():
+        raise ValueError("x must hold K and y N contiguous elements")
+    if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 32):
+        raise ValueError("q/s must be contiguous [N, K/2] / [N, K/32]")
+    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    _check("mxfp4_gemv_ex", lib.mxfp4_gemv_ex(_ptr(x), _ptr(q), _ptr(s), _ptr(y), N, K, flags, _stream(stream)))

@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 
+#include "mxfp4.h"
 #include "nvfp4.h"
 #include "nvfp4_kernels.h"
 
@@ -184,6 +185,54 @@ nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s
   cudaError_t e;
   e = nvfp4::launch_gemv(x, q, s, g, y, N, K, sms, static_w, (cudaStream_t)stream);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "gemv launch");
+}
+
+nvfp4_status mxfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, uint8_t* s,
+                            nvfp4_stream_t stream) {
+  if (K <= 0 || K % 32 != 0) return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 32", (long long)K);
+  if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
+  if (N == 0) return NVFP4_OK;
+  if (!w || !q || !s) return fail(NVFP4_ERR_INVALID_ARG, "null tensor pointer");
+  if (ldw < K) return fail(NVFP4_ERR_INVALID_ARG, "ldw=%lld < K=%lld", (long long)ldw, (long long)K);
+  if (!aligned16(w) || !aligned16(q) || !aligned16(s) || ldw % 8 != 0)
+    return fail(NVFP4_ERR_ALIGNMENT, "w, q, s must be 16-byte aligned and ldw a multiple of 8");
+  const size_t wb = (size_t)((N - 1) * ldw + K) * 2, qb = (size_t)(N * K / 2), sb = (size_t)(N * K / 32);
+  if (overlaps(w, wb, q, qb) || overlaps(w, wb, s, sb) || overlaps(q, qb, s, sb))
+    return fail(NVFP4_ERR_INVALID_ARG, "w, q and s must not overlap");
+  int sms = 0;
+  nvfp4_status st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_mx_quantize(w, N, K, ldw, q, s, (cudaStream_t)stream, sms);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "mxfp4 quantize launch");
+}
+
+nvfp4_status mxfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
+                        int64_t K, nvfp4_stream_t stream) {
+  return mxfp4_gemv_ex(x, q, s, y, N, K, 0u, stream);
+}
+
+nvfp4_status mxfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
+                           int64_t K, uint32_t flags, nvfp4_stream_t stream) {
+  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (K <= 0 || K % 32 != 0) return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 32", (long long)K);
+  if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
+  if (K > nvfp4::kGemvMaxK) return fail(NVFP4_ERR_SHAPE, "K=%lld exceeds the GEMV limit %lld", (long long)K, (long long)nvfp4::kGemvMaxK);
+  if (N > (int64_t)0x3FFFFFFF) return fail(NVFP4_ERR_SHAPE, "N=%lld too large", (long long)N);
+  if (N == 0) return NVFP4_OK;
+  if (!x || !q || !s || !y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(x) || !aligned16(q) || !aligned16(s))
+    return fail(NVFP4_ERR_ALIGNMENT, "x, q, s must be 16-byte aligned");
+  if (!aligned2(y)) return fail(NVFP4_ERR_ALIGNMENT, "y must be 2-byte aligned");
+  const size_t yb = (size_t)N * 2;
+  if (overlaps(y, yb, x, (size_t)K * 2) || overlaps(y, yb, q, (size_t)(N * K / 2)) ||
+      overlaps(y, yb, s, (size_t)(N * K / 32)))
+    return fail(NVFP4_ERR_INVALID_ARG, "y must not overlap x, q or s");
+  int sms = 0;
+  nvfp4_status st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  const bool static_w = (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0;
+  cudaError_t e = nvfp4::launch_gemv_mx(x, q, s, y, N, K, sms, static_w, (cudaStream_t)stream);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "mxfp4 gemv launch");
 }
 
 size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {

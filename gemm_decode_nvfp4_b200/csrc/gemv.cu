@@ -103,7 +103,59 @@ __device__ __noinline__ void gemv_rows_exact(const uint16_t* __restrict__ x, con
   }
 }
 
-template <int R, int CB, int MINB>
+// UE8M0 micro-scale (MXFP4) -> fp32: 2^(b - 127); 0 is the subnormal 2^-127,
+// 255 is NaN.
+__device__ __forceinline__ float e8m0_to_float(uint32_t b) {
+  return __uint_as_float(b == 0u ? 0x00400000u : (b == 255u ? 0x7FFFFFFFu : b << 23));
+}
+
+// MXFP4 counterpart of gemv_rows_exact: 32-element blocks with a UE8M0 scale,
+// no tensor scale.
+__device__ __noinline__ void gemv_rows_exact_mx(const uint16_t* __restrict__ x, const uint8_t* __restrict__ q,
+                                                const uint8_t* __restrict__ s, uint16_t* __restrict__ y, int N,
+                                                int K, int row0, int nrows) {
+  const int lane = threadIdx.x & 31;
+  for (int r = 0; r < nrows; ++r) {
+    const int row = row0 + r;
+    if (row >= N) break;
+    const uint8_t* qr = q + (int64_t)row * (K / 2);
+    const uint8_t* sr = s + (int64_t)row * (K / 32);
+    float acc = 0.0f;
+    for (int b = lane; b < K / 32; b += 32) {  // 32-element blocks
+      const uint4 w = *reinterpret_cast<const uint4*>(qr + 16 * b);
+      const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+      float2 p = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 xa = *reinterpret_cast<const uint4*>(x + 32 * b + 8 * i);
+        const uint32_t xw[4] = {xa.x, xa.y, xa.z, xa.w};
+        p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<0>(wd[i])), make_float2(bf16lo_to_float(xw[0]), bf16hi_to_float(xw[0])), p);
+        p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<1>(wd[i])), make_float2(bf16lo_to_float(xw[1]), bf16hi_to_float(xw[1])), p);
+        p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<2>(wd[i])), make_float2(bf16lo_to_float(xw[2]), bf16hi_to_float(xw[2])), p);
+        p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<3>(wd[i])), make_float2(bf16lo_to_float(xw[3]), bf16hi_to_float(xw[3])), p);
+      }
+      acc = fmaf(p.x + p.y, e8m0_to_float(sr[b]), acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    if (lane == 0) {
+      const __nv_bfloat16 o = __float2bfloat16_rn(acc);
+      y[row] = *reinterpret_cast<const uint16_t*>(&o);
+    }
+  }
+}
+
+// Rows row0 .. row0 + nrows - 1 exactly, in either format.
+template <bool MX>
+__device__ __forceinline__ void rows_exact(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
+                                           uint16_t* y, int N, int K, int row0, int nrows) {
+  if constexpr (MX)
+    gemv_rows_exact_mx(x, q, s, y, N, K, row0, nrows);
+  else
+    gemv_rows_exact(x, q, s, *g, y, N, K, row0, nrows);
+}
+
+template <int R, int CB, int MINB, bool MX>
 __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __restrict__ x,
                                                               const uint8_t* __restrict__ q,
                                                               const uint8_t* __restrict__ s,
@@ -116,8 +168,9 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   constexpr int kWords = CB / 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = (blockIdx.x * kWarps + warp) * R;
+  static_assert(!MX || CB == 16, "MXFP4: one 32-element block per 16-byte chunk");
   const int row_bytes = K >> 1;
-  const int row_scales = K >> 4;
+  const int row_scales = MX ? K >> 5 : K >> 4;
   const int steps = (row_bytes + 32 * CB - 1) / (32 * CB);
 
   auto load = [&](int step, uint32_t (&wq)[R][kWords], uint32_t (&ws)[R]) {
@@ -127,11 +180,11 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
       const int row = row0 + r;
       if (row < N && off < row_bytes) {
         const uint8_t* pq = q + (int64_t)row * row_bytes + off;
-        const uint8_t* ps = s + (int64_t)row * row_scales + off / 8;
+        const uint8_t* ps = s + (int64_t)row * row_scales + (MX ? off / 16 : off / 8);
         if constexpr (CB == 16) {
           const uint4 v = ld_stream_v4(pq);
           wq[r][0] = v.x; wq[r][1] = v.y; wq[r][2] = v.z; wq[r][3] = v.w;
-          ws[r] = *reinterpret_cast<const uint16_t*>(ps);
+          ws[r] = MX ? (uint32_t)*ps : (uint32_t)*reinterpret_cast<const uint16_t*>(ps);
         } else {
           const uint2 v = ld_stream_v2(pq);
           wq[r][0] = v.x; wq[r][1] = v.y;
@@ -187,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   }
 
   if (!fast) {  // x outside the f16 window: every warp takes its rows exactly
-    gemv_rows_exact(x, q, s, *g, y, N, K, row0, R);
+    rows_exact<MX>(x, q, s, g, y, N, K, row0, R);
     return;
   }
 
@@ -240,9 +293,13 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const float2 sc = f16x2_to_float2(e4m3x2_to_f16x2(cs[r]));
-      acc[r] = fmaf(part[r][0], sc.x, acc[r]);
-      if constexpr (kBlocks == 2) acc[r] = fmaf(part[r][1], sc.y, acc[r]);
+      if constexpr (MX) {
+        acc[r] = fmaf(part[r][0] + part[r][1], e8m0_to_float(cs[r]), acc[r]);
+      } else {
+        const float2 sc = f16x2_to_float2(e4m3x2_to_f16x2(cs[r]));
+        acc[r] = fmaf(part[r][0], sc.x, acc[r]);
+        if constexpr (kBlocks == 2) acc[r] = fmaf(part[r][1], sc.y, acc[r]);
+      }
     }
   };
   // Two register buffers in turn (the loop is unrolled by two so that no
@@ -258,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   }
   if (step < steps) compute(step, wq, ws);
 
-  const float gv = *g;
+  const float gv = MX ? 1.0f : *g;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     float v = acc[r];
@@ -280,11 +337,11 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   }
 }
 
-template <int R, int CB, int MINB>
+template <int R, int CB, int MINB, bool MX>
 cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y, int N,
                    int K, bool static_weights, cudaStream_t stream) {
   const size_t smem = (size_t)K * sizeof(uint16_t);
-  auto kern = gemv_kernel<R, CB, MINB>;
+  auto kern = gemv_kernel<R, CB, MINB, MX>;
   static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -340,12 +397,14 @@ __device__ __forceinline__ void tma_load_2d_evict_first(void* dst, const void* t
 // 128 contiguous bytes), then the barriers and the reduction scratch.
 // Rows of a CTA: [blockIdx.x * nblk * BR, + nblk * BR), in nblk blocks of BR
 // rows (BR <= 120) that go through the ring one 256-byte column at a time.
+template <bool MX>
 __global__ void __launch_bounds__(kRingThreads, 2)
     gemv_ring_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
                      const uint16_t* __restrict__ x, const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
                      const float* __restrict__ g, uint16_t* __restrict__ y, int N, int K, int BR, int nblk,
                      int S) {
   extern __shared__ __align__(1024) uint8_t sm[];
+  constexpr int kSB = MX ? kRingBK / 16 : kRingBK / 8;  // scale bytes of a row per stage
   const int nks = (K / 2 + kRingBK - 1) / kRingBK;  // stages per row block
   uint8_t* ring = sm;
   uint4* xs = reinterpret_cast<uint4*>(sm + S * kRingStage);
@@ -382,9 +441,9 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     auto issue = [&]() {
       uint8_t* dst = ring + slot * kRingStage;
       const int row0 = row_base + rb * BR;
-      ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)BR * (kRingBK + kRingBK / 8));
+      ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)BR * (kRingBK + kSB));
       tma_load_2d_evict_first(dst, &tq, &full[slot], t * kRingBK, row0, policy);
-      tma_load_2d_evict_first(dst + kRingScOff, &ts, &full[slot], t * (kRingBK / 8), row0, policy);
+      tma_load_2d_evict_first(dst + kRingScOff, &ts, &full[slot], t * kSB, row0, policy);
       if (++slot == S) { slot = 0; phase ^= 1; }
       if (++t == nks) { t = 0; ++rb; }
     };
@@ -453,11 +512,11 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     e = 15 - hi_exp;
     fast = hi_exp - lo_exp <= 32;
   }
-  const float gv = *g;
+  const float gv = MX ? 1.0f : *g;
   if (!fast) {  // x outside the f16 window: the producer stops, every warp takes rows exactly
     *abort_flag = 1;
     const int nrows = min(N - row_base, nblk * BR);
-    for (int r = warp; r < nrows; r += kRingConsumerWarps) gemv_rows_exact(x, q, s, gv, y, N, K, row_base + r, 1);
+    for (int r = warp; r < nrows; r += kRingConsumerWarps) rows_exact<MX>(x, q, s, g, y, N, K, row_base + r, 1);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     return;
   }
@@ -490,7 +549,7 @@ __global__ void __launch_bounds__(kRingThreads, 2)
   const int c = tid & (kRingChunks - 1);
   const int r0 = (tid / kRingChunks) * kRingRows;
   const uint8_t* lane_codes = ring + r0 * kRingBK + c * 16;
-  const uint8_t* lane_scales = ring + kRingScOff + r0 * (kRingBK / 8) + 2 * c;
+  const uint8_t* lane_scales = ring + kRingScOff + r0 * kSB + (MX ? c : 2 * c);
   const uint4* lane_x = xs + c;
   int slot = 0;
   uint32_t phase = 0;
@@ -509,7 +568,7 @@ __global__ void __launch_bounds__(kRingThreads, 2)
 #pragma unroll
       for (int i = 0; i < kRingRows; ++i) {
         cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingBK);
-        sc[i] = *reinterpret_cast<const uint16_t*>(ps + i * (kRingBK / 8));
+        sc[i] = MX ? (uint32_t)ps[i * kSB] : (uint32_t)*reinterpret_cast<const uint16_t*>(ps + i * kSB);
       }
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&empty[slot]);  // the stage's bytes are in registers
@@ -534,9 +593,13 @@ __global__ void __launch_bounds__(kRingThreads, 2)
       }
 #pragma unroll
       for (int i = 0; i < kRingRows; ++i) {
-        const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
-        acc[i] = fmaf(part[i][0], sf.x, acc[i]);
-        acc[i] = fmaf(part[i][1], sf.y, acc[i]);
+        if constexpr (MX) {  // one 32-element block per chunk
+          acc[i] = fmaf(part[i][0] + part[i][1], e8m0_to_float(sc[i]), acc[i]);
+        } else {
+          const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
+          acc[i] = fmaf(part[i][0], sf.x, acc[i]);
+          acc[i] = fmaf(part[i][1], sf.y, acc[i]);
+        }
       }
     }
 #pragma unroll
@@ -565,8 +628,9 @@ struct RingPlan {
 
 // The ring kernel's shape: rows split evenly over the SMs, shared memory for at
 // least two stages within half of the SM.  False when K does not fit it.
-bool ring_plan(int64_t N, int64_t K, int sms, RingPlan& p) {
-  if (K % 256 != 0 || K > kRingMaxK || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
+bool ring_plan(int64_t N, int64_t K, int sms, bool mx, RingPlan& p) {
+  // TMA row strides are multiples of 16 bytes: K/16 (NVFP4) or K/32 (MXFP4) scale bytes
+  if (K % (mx ? 512 : 256) != 0 || K > kRingMaxK || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
   int dev = 0, per_sm = 0, reserved = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
@@ -585,26 +649,28 @@ bool ring_plan(int64_t N, int64_t K, int sms, RingPlan& p) {
   return true;
 }
 
+template <bool MX>
 cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
                         int64_t N, int64_t K, cudaStream_t stream, const RingPlan& p, bool* encoded) {
   CUtensorMap tq, ts;
+  const int64_t sbytes = MX ? K / 32 : K / 16;  // scale bytes per row
   *encoded = tc::make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, N, K / 2, kRingBK, p.BR,
                               CU_TENSOR_MAP_SWIZZLE_NONE) &&
-             tc::make_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, K / 16, N, K / 16, kRingBK / 8, p.BR,
-                              CU_TENSOR_MAP_SWIZZLE_NONE);
+             tc::make_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, sbytes, N, sbytes,
+                              MX ? kRingBK / 16 : kRingBK / 8, p.BR, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!*encoded) return cudaSuccess;
   static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || smem_set[dev] < (int)p.smem) {
-    e = cudaFuncSetAttribute(gemv_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    e = cudaFuncSetAttribute(gemv_ring_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) smem_set[dev] = (int)p.smem;
   }
   int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S;
   void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S};
-  return tc::launch_pdl((const void*)gemv_ring_kernel, dim3(p.grid), dim3(kRingThreads), p.smem, stream, args);
+  return tc::launch_pdl((const void*)gemv_ring_kernel<MX>, dim3(p.grid), dim3(kRingThreads), p.smem, stream, args);
 }
 
 }  // namespace
@@ -612,13 +678,24 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream) {
   RingPlan plan;
-  if (ring_plan(N, K, sms, plan)) {
+  if (ring_plan(N, K, sms, false, plan)) {
     bool encoded = false;
-    const cudaError_t e = launch_ring(x, q, s, g, y, N, K, stream, plan, &encoded);
+    const cudaError_t e = launch_ring<false>(x, q, s, g, y, N, K, stream, plan, &encoded);
     if (encoded || e != cudaSuccess) return e;
   }
-  if (K % 32 == 0) return launch<8, 16, 2>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
-  return launch<8, 8, 2>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
+  if (K % 32 == 0) return launch<8, 16, 2, false>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
+  return launch<8, 8, 2, false>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
+}
+
+cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
+                           int64_t K, int sms, bool static_weights, cudaStream_t stream) {
+  RingPlan plan;
+  if (ring_plan(N, K, sms, true, plan)) {
+    bool encoded = false;
+    const cudaError_t e = launch_ring<true>(x, q, s, nullptr, y, N, K, stream, plan, &encoded);
+    if (encoded || e != cudaSuccess) return e;
+  }
+  return launch<8, 16, 2, true>(x, q, s, nullptr, y, (int)N, (int)K, static_weights, stream);
 }
 
 cudaError_t read_and_clear_gemv_timeouts(unsigned int* count) {

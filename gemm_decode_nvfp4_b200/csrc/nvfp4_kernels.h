@@ -22,6 +22,13 @@ cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream);
 // (programmatic dependent launch).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream);
+// MXFP4 decode GEMV (gemv.cu): one UE8M0 scale per 32 elements, no tensor
+// scale; K a multiple of 32.
+cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
+                           int64_t K, int sms, bool static_weights, cudaStream_t stream);
+// MXFP4 round-to-nearest quantizer (quantize.cu); K a multiple of 32.
+cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, uint8_t* s,
+                               cudaStream_t stream, int sms);
 // CTAs of the decode GEMV whose bounded pipeline wait gave up since the last read.
 cudaError_t read_and_clear_gemv_timeouts(unsigned int* count);
 

@@ -161,6 +161,68 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint16_t* __restric
   }
 }
 
+// ---------------------------------------------------------------------- MXFP4
+//
+// imp docs/quantization.md, MXFP4 paragraph: the NVFP4 nibble layout with one
+// UE8M0 (power-of-two) micro-scale per 32 elements and no tensor scale,
+// quantized round-to-nearest.  Scale rule (the pages give none; this is the
+// shared-exponent rule of the microscaling convention): X = 2^(floor(log2
+// amax_b) - 2), so the block maximum lands in [4, 8) before rounding and 6
+// clips it; byte = that exponent + 127, at least 0.  For a finite amax with
+// biased fp32 exponent field ef, floor(log2 amax) = ef - 127 when ef > 0, so
+// byte = max(ef - 2, 0), and zero or subnormal maxima give byte 0.
+// Elements are multiplied by 2^(127 - byte), a normal fp32 for every byte
+// 0..252 (exact), and rounded to E2M1 by the same RNE, saturating, sign-keeping
+// conversion as NVFP4.
+
+// One 32-element block: 16 code bytes and the UE8M0 byte.
+__device__ __forceinline__ void mx_quantize_store(const uint4 (&v)[4], uint8_t* qd, uint8_t* sd) {
+  float f[32];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[8 * j + 2 * i] = bf16lo_to_float(w4[i]);
+      f[8 * j + 2 * i + 1] = bf16hi_to_float(w4[i]);
+    }
+  }
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax_b = fmaxf(amax_b, fabsf(f[i]));
+  const uint32_t ef = (__float_as_uint(amax_b) >> 23) & 0xFFu;
+  const uint32_t byte = ef >= 2u ? ef - 2u : 0u;
+  const float m = __uint_as_float((254u - byte) << 23);  // 2^(127 - byte)
+  uint32_t c[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) c[i] = float2_to_e2m1x2_satfinite(__fmul_rn(f[2 * i], m), __fmul_rn(f[2 * i + 1], m));
+  uint4 codes;
+  codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+  codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+  codes.z = c[8] | (c[9] << 8) | (c[10] << 16) | (c[11] << 24);
+  codes.w = c[12] | (c[13] << 8) | (c[14] << 16) | (c[15] << 24);
+  *reinterpret_cast<uint4*>(qd) = codes;
+  *sd = static_cast<uint8_t>(byte);
+}
+
+// Thread t owns 32-element blocks t, t + stride, ...: 64 bytes in (four 16-byte
+// loads), 16 code bytes and one scale byte out.
+__global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t K,
+                                                          int64_t ldw, uint8_t* __restrict__ q,
+                                                          uint8_t* __restrict__ s) {
+  const int64_t bpr = K / 32;
+  const int64_t total = N * bpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
+    const int64_t n = ldw == K ? 0 : t / bpr, b = ldw == K ? t : t - n * bpr;
+    const uint4* src = reinterpret_cast<const uint4*>(w + n * ldw + b * 32);
+    uint4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = ld_stream_v4(src + j);
+    mx_quantize_store(v, q + t * 16, s + t);
+  }
+}
+
 __global__ void finalize_scale_kernel(float* amax_then_g) {
   *amax_then_g = __fdiv_rn(*amax_then_g, 2688.0f);
 }
@@ -185,6 +247,13 @@ cudaError_t launch_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw
                             cudaStream_t stream, int sms) {
   const int grid = grid_for(N * (K / 16), sms);
   quantize_kernel<<<grid, 256, 0, stream>>>(w, N, K, ldw, amax, q, s, g_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, uint8_t* s,
+                               cudaStream_t stream, int sms) {
+  const int grid = grid_for(N * (K / 32), sms);
+  mx_quantize_kernel<<<grid, 256, 0, stream>>>(w, N, K, ldw, q, s);
   return cudaGetLastError();
 }
 

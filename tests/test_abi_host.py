@@ -77,3 +77,21 @@ def test_unknown_flags_rejected():
     assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 4, 64, 0x80, None) == INVALID
     assert nv.lib.nvfp4_gemm_ex(A, 64, A, A, A, A + 4096, 64, 4, 64, 64, None, 0, 0x2, None) == INVALID
     assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 0, 64, 1, None) == OK   # N == 0: no-op
+
+
+def test_mxfp4_exports_and_validation():
+    names = set(nv.declared_symbols())
+    assert {"mxfp4_quantize", "mxfp4_gemv", "mxfp4_gemv_ex"} <= names
+    for K in (0, 16, 48, -32):
+        assert nv.lib.mxfp4_quantize(A, 4, K, 64, A + 4096, A + 8192, None) == SHAPE
+        assert nv.lib.mxfp4_gemv(A, A, A, A + 4096, 4, K, None) == SHAPE
+    assert b"multiple of 32" in nv.lib.nvfp4_last_error()
+    assert nv.lib.mxfp4_quantize(A, 0, 64, 64, A, A, None) == OK              # no-op
+    assert nv.lib.mxfp4_quantize(A, 4, 64, 32, A + 4096, A + 8192, None) == INVALID   # ldw < K
+    assert nv.lib.mxfp4_quantize(A, 4, 64, 64, A + 16, A + 8192, None) == INVALID     # q inside w
+    assert nv.lib.mxfp4_quantize(A, 4, 64, 64, A + 4096, A + 8200, None) == ALIGN
+    assert nv.lib.mxfp4_gemv(A, A, A, A, 0, 64, None) == OK
+    assert nv.lib.mxfp4_gemv(None, A, A, A, 4, 64, None) == INVALID
+    assert nv.lib.mxfp4_gemv(A + 8, A, A, A + 4096, 4, 64, None) == ALIGN
+    assert nv.lib.mxfp4_gemv(A, A + 8192, A + 16384, A + 16, 4, 64, None) == INVALID  # y overlaps x
+    assert nv.lib.mxfp4_gemv_ex(A, A, A, A + 4096, 4, 64, 2, None) == INVALID         # unknown flag
