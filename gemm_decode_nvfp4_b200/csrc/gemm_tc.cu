@@ -195,24 +195,44 @@ __device__ float exact_row_dot(const uint8_t* __restrict__ q, const uint8_t* __r
 // info[m] = e_m, or kWideRow when the row is not finite or its non-zero
 // magnitudes span more than 2^32 (then X' is not exact and the GEMM recomputes
 // the row on CUDA cores).
-__global__ void __launch_bounds__(128) prep_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int K,
-                                                     int* __restrict__ info, uint16_t* __restrict__ Xh) {
-  __shared__ uint32_t red_max[4], red_min[4];
+constexpr int kPrepThreads = 256;
+constexpr int kPrepPer = 8;  // 16-byte vectors per thread held in registers (K <= 256 * 8 * 8 = 16384)
+
+// Row m of X: range of |x| and X'[m, :] = f16(X[m, :] * 2^e_m).  For K <= 16384
+// every thread issues all of its loads at once and keeps the values in
+// registers for the conversion (one memory round trip); longer rows read X
+// twice.
+__global__ void __launch_bounds__(kPrepThreads) prep_x_kernel(const uint16_t* __restrict__ X, int64_t ldx, int K,
+                                                              int* __restrict__ info, uint16_t* __restrict__ Xh) {
+  __shared__ uint32_t red_max[kPrepThreads / 32], red_min[kPrepThreads / 32];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int m = blockIdx.x;
   const uint16_t* xr = X + (int64_t)m * ldx;
   uint16_t* hr = Xh + (int64_t)m * K;
+  const int nv = K / 8;
+  const bool in_regs = nv <= kPrepThreads * kPrepPer;
+  uint4 v[kPrepPer];
   uint32_t mx = 0, mn = 0xFFFFu;
-  for (int i = threadIdx.x; i < K / 8; i += 128) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xr + 8 * i);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  auto scan = [&](const uint4& x4) {
+    const uint32_t w4[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
       mx = max(mx, max(lo, hi));
       mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
     }
+  };
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kPrepPer; ++k) {
+      const int i = threadIdx.x + k * kPrepThreads;
+      v[k] = i < nv ? *reinterpret_cast<const uint4*>(xr + 8 * i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < kPrepPer; ++k) scan(v[k]);
+  } else {
+    for (int i = threadIdx.x; i < nv; i += kPrepThreads) scan(*reinterpret_cast<const uint4*>(xr + 8 * i));
   }
   mx = __reduce_max_sync(0xFFFFFFFFu, mx);
   mn = __reduce_min_sync(0xFFFFFFFFu, mn);
@@ -221,8 +241,13 @@ __global__ void __launch_bounds__(128) prep_x_kernel(const uint16_t* __restrict_
     red_min[threadIdx.x >> 5] = mn;
   }
   __syncthreads();
-  mx = max(max(red_max[0], red_max[1]), max(red_max[2], red_max[3]));
-  mn = min(min(red_min[0], red_min[1]), min(red_min[2], red_min[3]));
+  mx = red_max[0];
+  mn = red_min[0];
+#pragma unroll
+  for (int w = 1; w < kPrepThreads / 32; ++w) {
+    mx = max(mx, red_max[w]);
+    mn = min(mn, red_min[w]);
+  }
   int e = 0;
   bool wide = false;
   if (mx >= 0x7F80u) {
@@ -234,16 +259,25 @@ __global__ void __launch_bounds__(128) prep_x_kernel(const uint16_t* __restrict_
   }
   const int e1 = e / 2, e2 = e - e1;
   const float m1 = exp2i(e1), m2 = exp2i(e2);
-  for (int i = threadIdx.x; i < K / 8; i += 128) {
-    const uint4 v = *reinterpret_cast<const uint4*>(xr + 8 * i);
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  auto convert = [&](const uint4& x4) {
+    const uint32_t w4[4] = {x4.x, x4.y, x4.z, x4.w};
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const __half2 h = __floats2half2_rn(bf16lo_to_float(w4[j]) * m1 * m2, bf16hi_to_float(w4[j]) * m1 * m2);
       o[j] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    *reinterpret_cast<uint4*>(hr + 8 * i) = make_uint4(o[0], o[1], o[2], o[3]);
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  if (in_regs) {
+#pragma unroll
+    for (int k = 0; k < kPrepPer; ++k) {
+      const int i = threadIdx.x + k * kPrepThreads;
+      if (i < nv) *reinterpret_cast<uint4*>(hr + 8 * i) = convert(v[k]);
+    }
+  } else {
+    for (int i = threadIdx.x; i < nv; i += kPrepThreads)
+      *reinterpret_cast<uint4*>(hr + 8 * i) = convert(*reinterpret_cast<const uint4*>(xr + 8 * i));
   }
   if (threadIdx.x == 0) info[m] = wide ? kWideRow : e;
 }
@@ -616,7 +650,7 @@ cudaError_t launch_gemm_prep(const uint16_t* X, int64_t ldx, int64_t M, int64_t 
   const uint16_t* xp = X;
   int kk = (int)K;
   void* args[] = {(void*)&xp, &ldx, &kk, (void*)&info, (void*)&Xh};
-  return launch_pdl((const void*)prep_x_kernel, dim3((unsigned)M), dim3(128), 0, stream, args);
+  return launch_pdl((const void*)prep_x_kernel, dim3((unsigned)M), dim3(kPrepThreads), 0, stream, args);
 }
 
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,
