@@ -241,3 +241,29 @@ def mx_linear(x, q: np.ndarray, s: np.ndarray, rows=None, cols=None):
     lib().oracle_mx_linear(_ptr(xb), K, _ptr(q), _ptr(s), M, N, K, _ptr(ri), _ptr(ci), len(ri),
                            _ptr(y), _ptr(bound))
     return y, bound
+
+
+# ------------------------------------------------------ grouped (MoE) GEMV
+
+def linear_grouped(X, q: np.ndarray, s: np.ndarray, g: np.ndarray, expert_ids, token_ids):
+    """Grouped decode GEMV over stacked experts (imp docs/quantization.md, MoE
+    layers: one contiguous [ne, N, K_packed] buffer per projection, per-expert
+    scales).  For problem p: y[p] = x[token_ids[p]] . W[expert_ids[p]]^T with
+    expert e's codes q[e], scales s[e] and tensor scale g[e].  Returns
+    (y [P, N], bound [P, N]) in fp64, each row from ``linear``."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    g = np.asarray(g, np.float32).reshape(-1)
+    xb = _bf16_bits(X)
+    if xb.ndim == 1:
+        xb = xb.reshape(1, -1)
+    E, N = q.shape[0], q.shape[1]
+    ids_e = np.asarray(expert_ids, np.int64).reshape(-1)
+    ids_t = np.asarray(token_ids, np.int64).reshape(-1)
+    assert ids_e.shape == ids_t.shape and s.shape[:2] == (E, N) and g.shape == (E,)
+    y = np.empty((len(ids_e), N), np.float64)
+    bound = np.empty((len(ids_e), N), np.float64)
+    for p, (e, t) in enumerate(zip(ids_e, ids_t)):
+        yp, bp = linear(xb[t:t + 1], q[e], s[e], g[e])
+        y[p], bound[p] = yp[0], bp[0]
+    return y, bound
