@@ -22,7 +22,7 @@ __all__ = [
     "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
     "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
-    "mx_quantize", "mx_quantize_new", "mx_gemv",
+    "mx_quantize", "mx_quantize_new", "mx_gemv", "gemv_grouped",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -47,6 +47,8 @@ lib.nvfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _
 lib.nvfp4_gemm_ex.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_noalloc.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
+lib.nvfp4_gemv_grouped.argtypes = [_p, _i64, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64,
+                                   ctypes.c_uint32, _p]
 lib.mxfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p]
 lib.mxfp4_gemv.argtypes = [_p, _p, _p, _p, _i64, _i64, _p]
 lib.mxfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
@@ -54,7 +56,7 @@ lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
 for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
            lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors, lib.mxfp4_quantize, lib.mxfp4_gemv,
-           lib.mxfp4_gemv_ex):
+           lib.mxfp4_gemv_ex, lib.nvfp4_gemv_grouped):
     _f.restype = ctypes.c_int
 
 
@@ -284,3 +286,30 @@ def mx_gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, y: torch.Tensor, 
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/32]")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
     _check("mxfp4_gemv_ex", lib.mxfp4_gemv_ex(_ptr(x), _ptr(q), _ptr(s), _ptr(y), N, K, flags, _stream(stream)))
+
+
+# ------------------------------------------------------------ grouped (MoE) GEMV
+
+def gemv_grouped(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, expert_ids: torch.Tensor,
+                 token_ids: torch.Tensor, Y: torch.Tensor, stream=None) -> None:
+    """Y[p] = bf16(g[e] * W_deq[e] . X[t]) for e = expert_ids[p], t = token_ids[p]
+    with stacked experts q [E, N, K/2], s [E, N, K/16], g [E] (imp docs/quantization.md,
+    MoE layers: one contiguous [ne, N, K_packed] buffer per projection)."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(q, torch.uint8, "q", 3)
+    _need(s, torch.uint8, "s", 3)
+    _need(g, torch.float32, "g")
+    _need(expert_ids, torch.int32, "expert_ids")
+    _need(token_ids, torch.int32, "token_ids")
+    _need(Y, torch.bfloat16, "Y", 2)
+    E, N, K = q.shape[0], q.shape[1], q.shape[2] * 2
+    T, P = X.shape[0], expert_ids.numel()
+    if X.shape[1] != K or X.stride(1) != 1 or Y.stride(1) != 1 or Y.shape != (P, N):
+        raise ValueError("X must be [T, K] and Y [P, N] with unit column stride")
+    if not q.is_contiguous() or not s.is_contiguous() or s.shape != (E, N, K // 16) or g.numel() != E:
+        raise ValueError("q/s/g must be contiguous [E, N, K/2] / [E, N, K/16] / [E]")
+    if token_ids.numel() != P or not expert_ids.is_contiguous() or not token_ids.is_contiguous():
+        raise ValueError("expert_ids and token_ids must be contiguous [P]")
+    _check("nvfp4_gemv_grouped", lib.nvfp4_gemv_grouped(
+        _ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(expert_ids), _ptr(token_ids), _ptr(Y), Y.stride(0),
+        P, E, T, N, K, 0, _stream(stream)))

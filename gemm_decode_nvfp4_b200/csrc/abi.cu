@@ -187,6 +187,40 @@ nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "gemv launch");
 }
 
+nvfp4_status nvfp4_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                                const float* g, const int32_t* expert_ids, const int32_t* token_ids, uint16_t* Y,
+                                int64_t ldy, int64_t P, int64_t E, int64_t T, int64_t N, int64_t K, uint32_t flags,
+                                nvfp4_stream_t stream) {
+  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  nvfp4_status st = check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (P < 0 || E < 1 || T < 1 || N < 0)
+    return fail(NVFP4_ERR_SHAPE, "P=%lld E=%lld T=%lld N=%lld: need P >= 0, E >= 1, T >= 1, N >= 0", (long long)P,
+                (long long)E, (long long)T, (long long)N);
+  if (P > 65535) return fail(NVFP4_ERR_SHAPE, "P=%lld exceeds 65535 problems per call", (long long)P);
+  if (K > nvfp4::kGemvMaxK) return fail(NVFP4_ERR_SHAPE, "K=%lld exceeds the GEMV limit %lld", (long long)K, (long long)nvfp4::kGemvMaxK);
+  if (N > (int64_t)0x3FFFFFFF || E > (int64_t)0x7FFFFFFF || T > (int64_t)0x7FFFFFFF)
+    return fail(NVFP4_ERR_SHAPE, "N, E or T too large");
+  if (P == 0 || N == 0) return NVFP4_OK;
+  if (!X || !q || !s || !g || !expert_ids || !token_ids || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (ldx < K || ldy < N) return fail(NVFP4_ERR_INVALID_ARG, "ldx=%lld < K or ldy=%lld < N", (long long)ldx, (long long)ldy);
+  if (!aligned16(X) || ldx % 8 != 0 || !aligned16(q) || !aligned16(s))
+    return fail(NVFP4_ERR_ALIGNMENT, "X, q, s must be 16-byte aligned and ldx a multiple of 8");
+  if (!aligned2(Y) || !aligned4(g) || !aligned4(expert_ids) || !aligned4(token_ids))
+    return fail(NVFP4_ERR_ALIGNMENT, "Y needs 2-byte, g and the id arrays 4-byte alignment");
+  const size_t yb = (size_t)((P - 1) * ldy + N) * 2;
+  if (overlaps(Y, yb, X, (size_t)((T - 1) * ldx + K) * 2) || overlaps(Y, yb, q, (size_t)(E * N * K / 2)) ||
+      overlaps(Y, yb, s, (size_t)(E * N * K / 16)) || overlaps(Y, yb, g, (size_t)E * 4) ||
+      overlaps(Y, yb, expert_ids, (size_t)P * 4) || overlaps(Y, yb, token_ids, (size_t)P * 4))
+    return fail(NVFP4_ERR_INVALID_ARG, "Y must not overlap the inputs");
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_gemv_grouped(X, ldx, q, s, g, expert_ids, token_ids, Y, ldy, P, E, T, N, K, sms,
+                                             (cudaStream_t)stream);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "grouped gemv launch");
+}
+
 nvfp4_status mxfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, uint8_t* s,
                             nvfp4_stream_t stream) {
   if (K <= 0 || K % 32 != 0) return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 32", (long long)K);
@@ -315,9 +349,12 @@ nvfp4_status nvfp4_check_device_errors(void) {
   cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_small_timeouts(&k);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_timeouts(&v);
+  unsigned int bad = 0;
+  if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_bad_ids(&bad);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error counter");
   if (n || k || v)
     return fail(NVFP4_ERR_TIMEOUT, "%u GEMM, %u small-M GEMM and %u GEMV CTA(s) gave up on a pipeline wait", n, k, v);
+  if (bad) return fail(NVFP4_ERR_INVALID_ARG, "%u grouped GEMV problem(s) had an out-of-range expert or token id", bad);
   return NVFP4_OK;
 }
 

@@ -51,8 +51,47 @@ namespace nvfp4 {
 
 // CTAs of the ring kernel whose bounded pipeline wait gave up since the last read.
 __device__ unsigned int g_gemv_wait_timeouts = 0;
+// Grouped calls: problems whose expert or token id was out of range (their
+// output rows are written as zeros).
+__device__ unsigned int g_gemv_bad_ids = 0;
 
 namespace {
+
+// The problems of one launch: with expert_ids == nullptr a single GEMV (expert
+// 0, token 0); otherwise problem p = blockIdx.y multiplies expert
+// expert_ids[p] of the stacked [E, N, K/2] weights (and its tensor scale
+// g[e]) by row token_ids[p] of X into row p of Y (grouped MoE decode).
+struct Problems {
+  const int* expert_ids;
+  const int* token_ids;
+  int E, T;
+  int64_t x_stride, y_stride;  // elements between rows of X / of Y
+};
+
+// This CTA's expert and token; read only after griddepcontrol.wait (the ids
+// may come from the previous kernel).  False when an id is out of range.
+__device__ __forceinline__ bool resolve_problem(const Problems& P, int& e, int& tok) {
+  if (P.expert_ids == nullptr) {
+    e = 0;
+    tok = 0;
+    return true;
+  }
+  e = P.expert_ids[blockIdx.y];
+  tok = P.token_ids[blockIdx.y];
+  return e >= 0 && e < P.E && tok >= 0 && tok < P.T;
+}
+
+// Rows row0 .. row0 + nrows - 1 of an invalid problem become zeros (lane
+// first_thread, then every 32nd row); the problem is counted once, by thread 0
+// of its first CTA.
+__device__ __forceinline__ void zero_rows(uint16_t* y, int N, int row0, int nrows, int first_thread) {
+  for (int r = first_thread; r < nrows; r += 32)
+    if (row0 + r < N) y[row0 + r] = 0;
+}
+
+__device__ __forceinline__ void count_bad_problem() {
+  if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&g_gemv_bad_ids, 1u);
+}
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
@@ -161,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
                                                               const uint8_t* __restrict__ s,
                                                               const float* __restrict__ g,
                                                               uint16_t* __restrict__ y, int N, int K,
-                                                              int static_weights) {
+                                                              int static_weights, Problems P) {
   extern __shared__ __align__(16) uint8_t xsm[];  // K f16
   __shared__ uint32_t red_max[kWarps], red_min[kWarps];
   constexpr int kBlocks = (2 * CB) / 16;  // scales per lane-chunk (2 or 1)
@@ -202,10 +241,23 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   // its prologue; read the weights before the previous kernel has finished
   // only when the caller declared them static, x and y only after it has.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (!static_weights) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // grouped calls learn their expert only after the previous kernel
+  const bool early = static_weights && P.expert_ids == nullptr;
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
+  int e_id = 0, tok = 0;
+  if (!resolve_problem(P, e_id, tok)) {  // the warp's rows of this problem become zeros
+    zero_rows(y + (int64_t)blockIdx.y * P.y_stride, N, row0, R, lane);
+    count_bad_problem();
+    return;
+  }
+  q += (int64_t)e_id * N * (K / 2);
+  s += (int64_t)e_id * N * (MX ? K / 32 : K / 16);
+  if (!MX) g += e_id;
+  x += (int64_t)tok * P.x_stride;
+  y += (int64_t)blockIdx.y * P.y_stride;
   uint32_t wq[R][kWords], ws[R];
   load(0, wq, ws);  // first weights in flight before x is staged
-  if (static_weights) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---- range of |x| (bit patterns of non-negative BF16 order like values)
   uint32_t mx = 0, mn = 0xFFFFu;
@@ -339,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
 
 template <int R, int CB, int MINB, bool MX>
 cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y, int N,
-                   int K, bool static_weights, cudaStream_t stream) {
+                   int K, bool static_weights, cudaStream_t stream, const Problems& P, int num_problems) {
   const size_t smem = (size_t)K * sizeof(uint16_t);
   auto kern = gemv_kernel<R, CB, MINB, MX>;
   static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
@@ -354,7 +406,7 @@ cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const 
   const int rows_per_cta = kWarps * R;
   const int grid = (N + rows_per_cta - 1) / rows_per_cta;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3(grid, num_problems);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -363,7 +415,7 @@ cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, x, q, s, g, y, N, K, static_weights ? 1 : 0);
+  return cudaLaunchKernelEx(&cfg, kern, x, q, s, g, y, N, K, static_weights ? 1 : 0, P);
 }
 
 
@@ -383,12 +435,12 @@ constexpr uint64_t kRingWaitNs = 2000000000ull;
 
 __device__ __forceinline__ void ring_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
 
-__device__ __forceinline__ void tma_load_2d_evict_first(void* dst, const void* tmap, uint64_t* bar, int c0, int c1,
-                                                        uint64_t policy) {
+__device__ __forceinline__ void tma_load_3d_evict_first(void* dst, const void* tmap, uint64_t* bar, int c0, int c1,
+                                                        int c2, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(ptx::smem_u32(dst)),
-      "l"(tmap), "r"(ptx::smem_u32(bar)), "r"(c0), "r"(c1), "l"(policy)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(ptx::smem_u32(dst)),
+      "l"(tmap), "r"(ptx::smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
       : "memory");
 }
 
@@ -402,7 +454,7 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     gemv_ring_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
                      const uint16_t* __restrict__ x, const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
                      const float* __restrict__ g, uint16_t* __restrict__ y, int N, int K, int BR, int nblk,
-                     int S) {
+                     int S, Problems P) {
   extern __shared__ __align__(1024) uint8_t sm[];
   constexpr int kSB = MX ? kRingBK / 16 : kRingBK / 8;  // scale bytes of a row per stage
   const int nks = (K / 2 + kRingBK - 1) / kRingBK;  // stages per row block
@@ -436,20 +488,22 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     ptx::prefetch_tmap(&ts);
     uint64_t policy;  // each weight byte is read once: do not keep it in L2
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
-    int n = 0, slot = 0, t = 0, rb = 0;
+    int n = 0, slot = 0, t = 0, rb = 0, e_id = 0;
     uint32_t phase = 0;
     auto issue = [&]() {
       uint8_t* dst = ring + slot * kRingStage;
       const int row0 = row_base + rb * BR;
       ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)BR * (kRingBK + kSB));
-      tma_load_2d_evict_first(dst, &tq, &full[slot], t * kRingBK, row0, policy);
-      tma_load_2d_evict_first(dst + kRingScOff, &ts, &full[slot], t * kSB, row0, policy);
+      tma_load_3d_evict_first(dst, &tq, &full[slot], t * kRingBK, row0, e_id, policy);
+      tma_load_3d_evict_first(dst + kRingScOff, &ts, &full[slot], t * kSB, row0, e_id, policy);
       if (++slot == S) { slot = 0; phase ^= 1; }
       if (++t == nks) { t = 0; ++rb; }
     };
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // x and the weights only after this
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x, ids and the weights only after this
+    int tok = 0;
+    if (!resolve_problem(P, e_id, tok)) return;  // nothing issued: the consumers write zeros
     ptx::mbar_arrive_expect_tx(xfull, (uint32_t)K * 2);
-    ptx::bulk_load(xs, x, (uint32_t)K * 2, xfull);
+    ptx::bulk_load(xs, x + (int64_t)tok * P.x_stride, (uint32_t)K * 2, xfull);
     for (; n < total; ++n) {
       if (n >= S) {  // wait until the consumers have released this slot (or have given up on the ring)
         bool ok = ptx::mbar_try_wait(&empty[slot], phase ^ 1);
@@ -475,6 +529,20 @@ __global__ void __launch_bounds__(kRingThreads, 2)
 
   // ------------------------------------------------------------------------------- consumers
   asm volatile("griddepcontrol.wait;" ::: "memory");  // y is written only after the previous kernel
+  {
+    int e_id = 0, tok = 0;
+    if (!resolve_problem(P, e_id, tok)) {  // this CTA's rows of the problem become zeros
+      if (warp == 0)
+        for (int b = 0; b < nb_here; ++b) zero_rows(y + (int64_t)blockIdx.y * P.y_stride, N, row_base + b * BR, BR, lane);
+      count_bad_problem();
+      return;
+    }
+    q += (int64_t)e_id * N * (K / 2);
+    s += (int64_t)e_id * N * (MX ? K / 32 : K / 16);
+    if (!MX) g += e_id;
+    x += (int64_t)tok * P.x_stride;
+    y += (int64_t)blockIdx.y * P.y_stride;
+  }
   if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(xfull, 0, kRingWaitNs))) {
     if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
     *abort_flag = 1;
@@ -628,7 +696,7 @@ struct RingPlan {
 
 // The ring kernel's shape: rows split evenly over the SMs, shared memory for at
 // least two stages within half of the SM.  False when K does not fit it.
-bool ring_plan(int64_t N, int64_t K, int sms, bool mx, RingPlan& p) {
+bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, RingPlan& p) {
   // TMA row strides are multiples of 16 bytes: K/16 (NVFP4) or K/32 (MXFP4) scale bytes
   if (K % (mx ? 512 : 256) != 0 || K > kRingMaxK || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
   int dev = 0, per_sm = 0, reserved = 0;
@@ -636,7 +704,7 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, RingPlan& p) {
       cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
     return false;
-  const int64_t rpc = (N + sms - 1) / sms;
+  const int64_t rpc = ((int64_t)num_problems * N + sms - 1) / sms;  // rows of all problems over the SMs
   p.nblk = (int)((rpc + kRingMaxBR - 1) / kRingMaxBR);
   p.BR = (int)((rpc + p.nblk - 1) / p.nblk);
   p.grid = (int)((N + (int64_t)p.nblk * p.BR - 1) / ((int64_t)p.nblk * p.BR));
@@ -651,12 +719,14 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, RingPlan& p) {
 
 template <bool MX>
 cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
-                        int64_t N, int64_t K, cudaStream_t stream, const RingPlan& p, bool* encoded) {
-  CUtensorMap tq, ts;
+                        int64_t N, int64_t K, cudaStream_t stream, const RingPlan& p, const Problems& P,
+                        int num_problems, bool* encoded) {
+  CUtensorMap tq, ts;  // [E, N, K/2] codes and [E, N, scale bytes]: the expert is the third coordinate
   const int64_t sbytes = MX ? K / 32 : K / 16;  // scale bytes per row
-  *encoded = tc::make_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, N, K / 2, kRingBK, p.BR,
-                              CU_TENSOR_MAP_SWIZZLE_NONE) &&
-             tc::make_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, sbytes, N, sbytes,
+  const int64_t E = P.expert_ids ? P.E : 1;
+  *encoded = tc::make_tmap_3d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, K / 2, N, E, K / 2, N * (K / 2), kRingBK,
+                              p.BR, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             tc::make_tmap_3d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, sbytes, N, E, sbytes, N * sbytes,
                               MX ? kRingBK / 16 : kRingBK / 8, p.BR, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!*encoded) return cudaSuccess;
   static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
@@ -669,33 +739,58 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
     if (dev >= 0 && dev < 64) smem_set[dev] = (int)p.smem;
   }
   int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S;
-  void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S};
-  return tc::launch_pdl((const void*)gemv_ring_kernel<MX>, dim3(p.grid), dim3(kRingThreads), p.smem, stream, args);
+  Problems Pc = P;
+  void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S, &Pc};
+  return tc::launch_pdl((const void*)gemv_ring_kernel<MX>, dim3(p.grid, num_problems), dim3(kRingThreads), p.smem,
+                        stream, args);
 }
+
+}  // namespace
+
+namespace {
+
+template <bool MX>
+cudaError_t launch_any(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
+                       int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream, const Problems& P,
+                       int num_problems) {
+  RingPlan plan;
+  if (ring_plan(N, K, sms, MX, num_problems, plan)) {
+    bool encoded = false;
+    const cudaError_t e = launch_ring<MX>(x, q, s, g, y, N, K, stream, plan, P, num_problems, &encoded);
+    if (encoded || e != cudaSuccess) return e;
+  }
+  if (MX || K % 32 == 0)
+    return launch<8, 16, 2, MX>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
+  return launch<8, 8, 2, false>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
+}
+
+const Problems kSingle = {nullptr, nullptr, 1, 1, 0, 0};
 
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  RingPlan plan;
-  if (ring_plan(N, K, sms, false, plan)) {
-    bool encoded = false;
-    const cudaError_t e = launch_ring<false>(x, q, s, g, y, N, K, stream, plan, &encoded);
-    if (encoded || e != cudaSuccess) return e;
-  }
-  if (K % 32 == 0) return launch<8, 16, 2, false>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
-  return launch<8, 8, 2, false>(x, q, s, g, y, (int)N, (int)K, static_weights, stream);
+  return launch_any<false>(x, q, s, g, y, N, K, sms, static_weights, stream, kSingle, 1);
 }
 
 cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
                            int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  RingPlan plan;
-  if (ring_plan(N, K, sms, true, plan)) {
-    bool encoded = false;
-    const cudaError_t e = launch_ring<true>(x, q, s, nullptr, y, N, K, stream, plan, &encoded);
-    if (encoded || e != cudaSuccess) return e;
-  }
-  return launch<8, 16, 2, true>(x, q, s, nullptr, y, (int)N, (int)K, static_weights, stream);
+  return launch_any<true>(x, q, s, nullptr, y, N, K, sms, static_weights, stream, kSingle, 1);
+}
+
+cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                                const float* g, const int* expert_ids, const int* token_ids, uint16_t* Y,
+                                int64_t ldy, int64_t P, int64_t E, int64_t T, int64_t N, int64_t K, int sms,
+                                cudaStream_t stream) {
+  const Problems pr = {expert_ids, token_ids, (int)E, (int)T, ldx, ldy};
+  return launch_any<false>(X, q, s, g, Y, N, K, sms, false, stream, pr, (int)P);
+}
+
+cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count) {
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_gemv_bad_ids, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_gemv_bad_ids, &zero, sizeof(unsigned int));
 }
 
 cudaError_t read_and_clear_gemv_timeouts(unsigned int* count) {

@@ -26,6 +26,15 @@ cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
 // scale; K a multiple of 32.
 cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
                            int64_t K, int sms, bool static_weights, cudaStream_t stream);
+// Grouped (MoE) decode GEMV (gemv.cu): problem p multiplies expert expert_ids[p]
+// of the stacked weights q [E, N, K/2], s [E, N, K/16], g [E] by row
+// token_ids[p] of X [T, K] (leading dimension ldx) into row p of Y (ldy).
+cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                                const float* g, const int* expert_ids, const int* token_ids, uint16_t* Y,
+                                int64_t ldy, int64_t P, int64_t E, int64_t T, int64_t N, int64_t K, int sms,
+                                cudaStream_t stream);
+// Problems of grouped GEMVs whose ids were out of range since the last read.
+cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count);
 // MXFP4 round-to-nearest quantizer (quantize.cu); K a multiple of 32.
 cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, uint8_t* s,
                                cudaStream_t stream, int sms);

@@ -39,6 +39,21 @@ inline bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType type, const void*
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D row-major tensor [depth, outer, inner] (`row_bytes` between rows,
+// `plane_bytes` between planes), copied in boxes of [1, box_outer, box_inner].
+inline bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+                         uint64_t outer, uint64_t depth, uint64_t row_bytes, uint64_t plane_bytes,
+                         uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)depth};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)plane_bytes};
+  const cuuint32_t box[3] = {box_inner, box_outer, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, type, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel on the stream is finishing (it orders itself with
 // griddepcontrol.wait).

@@ -206,12 +206,33 @@ NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint16_t* X, int64_t ldx, const 
                                           int64_t K, uint32_t flags, nvfp4_stream_t stream);
 
 /*
+ * Grouped (MoE) decode GEMV over stacked experts ("MoE layers" pipeline of imp
+ * docs/quantization.md: one contiguous [ne, N, K_packed] buffer per layer and
+ * projection, read by the decode fast path).  For p = 0 .. P-1:
+ *   Y[p, n] = bf16_rn( g[e] * sum_j e4m3(s[e, n, j]) * sum_i e2m1(q[e, n, 16j+i]) * X[t, 16j+i] )
+ *   with e = expert_ids[p], t = token_ids[p].
+ * X: BF16 [T, K], leading dimension ldx (elements, multiple of 8); q: [E, N, K/2];
+ * s: [E, N, K/16]; g: fp32 [E] (each expert's own tensor scale); expert_ids,
+ * token_ids: device int32 [P] (e.g. written by a router kernel earlier on the
+ * stream: they are read after it completes); Y: BF16 [P, N], leading dimension
+ * ldy >= N.  A problem whose ids are out of range gets a zero output row and is
+ * counted for nvfp4_check_device_errors (NVFP4_ERR_INVALID_ARG).  P == 0 is a
+ * no-op; P <= 65535; K <= 49152.  flags: NVFP4_FLAG_* (the static-weights flag
+ * changes nothing here: the expert is known only after the previous kernel).
+ */
+NVFP4_API nvfp4_status nvfp4_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
+                                          const float* g, const int32_t* expert_ids, const int32_t* token_ids,
+                                          uint16_t* Y, int64_t ldy, int64_t P, int64_t E, int64_t T, int64_t N,
+                                          int64_t K, uint32_t flags, nvfp4_stream_t stream);
+
+/*
  * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMMs
  * and the TMA-fed decode GEMV) is bounded (about 2 s); a CTA that gives up
  * records it in a device counter and finishes without hanging, leaving its
  * outputs undefined.  This call reads and
  * clears that counter for the current device (it waits for prior work on the
- * legacy default stream) and returns NVFP4_ERR_TIMEOUT if it was non-zero.
+ * legacy default stream) and returns NVFP4_ERR_TIMEOUT if it was non-zero,
+ * else NVFP4_ERR_INVALID_ARG if grouped GEMVs met out-of-range ids.
  */
 NVFP4_API nvfp4_status nvfp4_check_device_errors(void);
 

@@ -95,3 +95,20 @@ def test_mxfp4_exports_and_validation():
     assert nv.lib.mxfp4_gemv(A + 8, A, A, A + 4096, 4, 64, None) == ALIGN
     assert nv.lib.mxfp4_gemv(A, A + 8192, A + 16384, A + 16, 4, 64, None) == INVALID  # y overlaps x
     assert nv.lib.mxfp4_gemv_ex(A, A, A, A + 4096, 4, 64, 2, None) == INVALID         # unknown flag
+
+
+def test_grouped_validation():
+    assert "nvfp4_gemv_grouped" in nv.declared_symbols()
+    f = nv.lib.nvfp4_gemv_grouped
+    # X, ldx, q, s, g, experts, tokens, Y, ldy, P, E, T, N, K, flags, stream
+    assert f(A, 64, A, A, A, A, A, A, 16, 0, 4, 1, 16, 64, 0, None) == OK           # P == 0: no-op
+    assert f(A, 64, A, A, A, A, A, A, 16, -1, 4, 1, 16, 64, 0, None) == SHAPE
+    assert f(A, 64, A, A, A, A, A, A, 16, 4, 0, 1, 16, 64, 0, None) == SHAPE        # E == 0
+    assert f(A, 64, A, A, A, A, A, A, 16, 70000, 4, 1, 16, 64, 0, None) == SHAPE    # too many problems
+    assert f(A, 64, A, A, A, A, A, A, 16, 4, 4, 1, 16, 24, 0, None) == SHAPE        # K % 16
+    assert f(A, 64, A, A, A, None, A, A + 8192, 16, 4, 4, 1, 16, 64, 0, None) == INVALID
+    assert f(A, 60, A, A, A, A, A, A + 8192, 16, 4, 4, 1, 16, 64, 0, None) == INVALID  # ldx < K
+    assert f(A, 68, A, A, A, A, A, A + 8192, 16, 4, 4, 1, 16, 64, 0, None) == ALIGN    # ldx % 8
+    assert f(A, 64, A, A, A, A + 2, A, A + 8192, 16, 4, 4, 1, 16, 64, 0, None) == ALIGN
+    assert f(A, 64, A + 8192, A + 16384, A + 24576, A + 32768, A + 32800, A, 16, 4, 4, 1, 16, 64, 0, None) == INVALID  # Y over X
+    assert f(A, 64, A, A, A, A, A, A + 8192, 16, 4, 4, 1, 16, 64, 4, None) == INVALID  # unknown flag
