@@ -61,6 +61,14 @@ def mx_quantize_bytes(N: int, K: int) -> int:
     return 2 * N * K + N * K // 2 + N * K // 32
 
 
+MOE = {"E": 128, "N": 1536, "K": 2048, "top": 8}  # synthetic MoE layer: stacked experts, top-8 routing, one token
+
+
+def moe_bytes(n_problems: int, N: int, K: int) -> int:
+    """Grouped decode GEMV: each problem's expert weights + x + y + ids and g."""
+    return n_problems * (N * K // 2 + N * K // 16 + 2 * N + 8 + 4) + 2 * K
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -91,6 +99,7 @@ KERNEL_SOURCES = {
     "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
     "mx_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
+    "moe_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
 }
 
 
@@ -266,6 +275,25 @@ def run_gpu(args):
     def mx_quant_all():
         nv.mx_quantize(wq_in, mq_out, ms_out)
 
+    # grouped MoE decode: 128 stacked experts [1536, 2048] (226 MB, more than L2),
+    # 8 calls per graph, each routing one token to 8 different experts
+    me, mn, mk, mtop = MOE["E"], MOE["N"], MOE["K"], MOE["top"]
+    moe_w = workloads.to_bf16(workloads.plain_weight_f32(me * mn, mk, 7)).to(dev)
+    moe_q, moe_s, _ = nv.quantize_new(moe_w)
+    del moe_w
+    moe_q = moe_q.reshape(me, mn, mk // 2)
+    moe_s = moe_s.reshape(me, mn, mk // 16)
+    moe_g = torch.full((me,), 0.004, dtype=torch.float32, device=dev)
+    moe_x = workloads.activations(1, mk, 5).to(dev)
+    route = torch.randperm(me, generator=torch.Generator().manual_seed(3))[: copies * mtop].reshape(copies, mtop)
+    moe_ids = route.to(torch.int32).to(dev)
+    moe_tok = torch.zeros((mtop,), dtype=torch.int32, device=dev)
+    moe_y = torch.empty((mtop, mn), dtype=torch.bfloat16, device=dev)
+
+    def moe_all():
+        for i in range(copies):
+            nv.gemv_grouped(moe_x, moe_q, moe_s, moe_g, moe_ids[i], moe_tok, moe_y)
+
     def quant_all():
         amax_buf.zero_()
         nv.amax(wq_in, amax_buf)
@@ -285,6 +313,7 @@ def run_gpu(args):
         rows.append(("gemm_m512", m512_all, copies, 2))
         rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
     rows.append(("mx_gemv", mx_gemv_all, copies, 1))
+    rows.append(("moe_gemv", moe_all, copies, 1))
     rows.append(("gemv_ordered", gemv_ordered_all, copies, 1))
     rows.append(("gemv", gemv_all, copies, 1))
     if args.only != "all":  # profiling runs: keep only the named row (plus the headline GEMV)
@@ -365,6 +394,12 @@ def run_gpu(args):
         kernels["mx_gemv"] = {"us": per_launch_ms["mx_gemv"] * 1e3, "GB/s": mg, "frac_hbm": mg / hbm, "bytes": mb,
                               "weight_bytes_per_token": N * K // 2 + N * K // 32,
                               "format": "MXFP4: UE8M0 scale per 32, no tensor scale"}
+    if "moe_gemv" in per_launch_ms:
+        mb = moe_bytes(MOE["top"], MOE["N"], MOE["K"])
+        mg = mb / (per_launch_ms["moe_gemv"] * 1e-3) / 1e9
+        kernels["moe_gemv"] = {"us": per_launch_ms["moe_gemv"] * 1e3, "GB/s": mg, "frac_hbm": mg / hbm, "bytes": mb,
+                               "workload": f"grouped decode GEMV: {MOE['top']} of {MOE['E']} stacked experts "
+                                           f"[{MOE['N']}, {MOE['K']}], one token, synthetic routing"}
     if "mx_quantize" in per_launch_ms:
         mb = mx_quantize_bytes(N, K)
         mq = mb / (per_launch_ms["mx_quantize"] * 1e-3) / 1e9
@@ -428,9 +463,9 @@ def run_gpu(args):
             "config": {"workload": WORKLOAD, "N": N, "K": K, "M": 1, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {copies} rotating weight copies "
                              f"({copies * (N * K // 2 + N * K // 16) / 1e6:.0f} MB) per graph",
-                       "row_order": "quantize, MXFP4 quantize, gemm M=512, gemm M=32, MXFP4 gemv, gemv ordered, gemv static: each GEMV graph "
+                       "row_order": "quantize, MXFP4 quantize, gemm M=512, gemm M=32, MXFP4 gemv, MoE gemv, gemv ordered, gemv static: each GEMV graph "
                                     "follows GEMVs, not the rows that leave tens of MB of dirty output in L2",
-                       "step": "quantize [17408,5120] (NVFP4, MXFP4) + gemm M=512 + gemm M=32 + MXFP4 gemv + gemv M=1 (x2: ordered and static-weights)",
+                       "step": "quantize [17408,5120] (NVFP4, MXFP4) + gemm M=512 + gemm M=32 + MXFP4 gemv + grouped MoE gemv + gemv M=1 (x2: ordered and static-weights)",
             "gemv_launch": "8 GEMVs per graph on 8 weight copies, programmatic dependent launch (static weights)"},
             "roofline": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemv_gbs / hbm, "traffic": traffic,
@@ -525,7 +560,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=17408)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "gemm_m32",
-                                                      "gemm_m512", "mx_gemv", "mx_quantize"],
+                                                      "gemm_m512", "mx_gemv", "mx_quantize", "moe_gemv"],
                     help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
