@@ -213,8 +213,24 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
   const int64_t bpr = K / 32;
   const int64_t total = N * bpr;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
-    const int64_t n = ldw == K ? 0 : t / bpr, b = ldw == K ? t : t - n * bpr;
+  int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (ldw == K) {
+    // contiguous rows: blocks t and t + stride together, eight 16-byte loads in flight
+    for (; t + stride < total; t += 2 * stride) {
+      const uint4* a = reinterpret_cast<const uint4*>(w + t * 32);
+      const uint4* b = reinterpret_cast<const uint4*>(w + (t + stride) * 32);
+      uint4 va[4], vb[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        va[j] = ld_stream_v4(a + j);
+        vb[j] = ld_stream_v4(b + j);
+      }
+      mx_quantize_store(va, q + t * 16, s + t);
+      mx_quantize_store(vb, q + (t + stride) * 16, s + t + stride);
+    }
+  }
+  for (; t < total; t += stride) {
+    const int64_t n = t / bpr, b = t - n * bpr;
     const uint4* src = reinterpret_cast<const uint4*>(w + n * ldw + b * 32);
     uint4 v[4];
 #pragma unroll
