@@ -70,8 +70,9 @@ struct Problems {
 
 // This CTA's expert and token; read only after griddepcontrol.wait (the ids
 // may come from the previous kernel).  False when an id is out of range.
+template <bool GROUPED>
 __device__ __forceinline__ bool resolve_problem(const Problems& P, int& e, int& tok) {
-  if (P.expert_ids == nullptr) {
+  if (!GROUPED || P.expert_ids == nullptr) {
     e = 0;
     tok = 0;
     return true;
@@ -194,7 +195,7 @@ __device__ __forceinline__ void rows_exact(const uint16_t* x, const uint8_t* q, 
     gemv_rows_exact(x, q, s, *g, y, N, K, row0, nrows);
 }
 
-template <int R, int CB, int MINB, bool MX>
+template <int R, int CB, int MINB, bool MX, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __restrict__ x,
                                                               const uint8_t* __restrict__ q,
                                                               const uint8_t* __restrict__ s,
@@ -242,10 +243,10 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   // only when the caller declared them static, x and y only after it has.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // grouped calls learn their expert only after the previous kernel
-  const bool early = static_weights && P.expert_ids == nullptr;
+  const bool early = static_weights && !GROUPED;
   if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
   int e_id = 0, tok = 0;
-  if (!resolve_problem(P, e_id, tok)) {  // the warp's rows of this problem become zeros
+  if (!resolve_problem<GROUPED>(P, e_id, tok)) {  // the warp's rows of this problem become zeros
     zero_rows(y + (int64_t)blockIdx.y * P.y_stride, N, row0, R, lane);
     count_bad_problem();
     return;
@@ -389,11 +390,11 @@ __global__ void __launch_bounds__(kThreads, MINB) gemv_kernel(const uint16_t* __
   }
 }
 
-template <int R, int CB, int MINB, bool MX>
+template <int R, int CB, int MINB, bool MX, bool GROUPED>
 cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y, int N,
                    int K, bool static_weights, cudaStream_t stream, const Problems& P, int num_problems) {
   const size_t smem = (size_t)K * sizeof(uint16_t);
-  auto kern = gemv_kernel<R, CB, MINB, MX>;
+  auto kern = gemv_kernel<R, CB, MINB, MX, GROUPED>;
   static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -449,7 +450,7 @@ __device__ __forceinline__ void tma_load_3d_evict_first(void* dst, const void* t
 // 128 contiguous bytes), then the barriers and the reduction scratch.
 // Rows of a CTA: [blockIdx.x * nblk * BR, + nblk * BR), in nblk blocks of BR
 // rows (BR <= 120) that go through the ring one 256-byte column at a time.
-template <bool MX>
+template <bool MX, bool GROUPED>
 __global__ void __launch_bounds__(kRingThreads, 2)
     gemv_ring_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
                      const uint16_t* __restrict__ x, const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     };
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x, ids and the weights only after this
     int tok = 0;
-    if (!resolve_problem(P, e_id, tok)) return;  // nothing issued: the consumers write zeros
+    if (!resolve_problem<GROUPED>(P, e_id, tok)) return;  // nothing issued: the consumers write zeros
     ptx::mbar_arrive_expect_tx(xfull, (uint32_t)K * 2);
     ptx::bulk_load(xs, x + (int64_t)tok * P.x_stride, (uint32_t)K * 2, xfull);
     for (; n < total; ++n) {
@@ -531,7 +532,7 @@ __global__ void __launch_bounds__(kRingThreads, 2)
   asm volatile("griddepcontrol.wait;" ::: "memory");  // y is written only after the previous kernel
   {
     int e_id = 0, tok = 0;
-    if (!resolve_problem(P, e_id, tok)) {  // this CTA's rows of the problem become zeros
+    if (!resolve_problem<GROUPED>(P, e_id, tok)) {  // this CTA's rows of the problem become zeros
       if (warp == 0)
         for (int b = 0; b < nb_here; ++b) zero_rows(y + (int64_t)blockIdx.y * P.y_stride, N, row_base + b * BR, BR, lane);
       count_bad_problem();
@@ -717,7 +718,7 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, RingPla
   return true;
 }
 
-template <bool MX>
+template <bool MX, bool GROUPED>
 cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
                         int64_t N, int64_t K, cudaStream_t stream, const RingPlan& p, const Problems& P,
                         int num_problems, bool* encoded) {
@@ -734,14 +735,14 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || smem_set[dev] < (int)p.smem) {
-    e = cudaFuncSetAttribute(gemv_ring_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    e = cudaFuncSetAttribute(gemv_ring_kernel<MX, GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) smem_set[dev] = (int)p.smem;
   }
   int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S;
   Problems Pc = P;
   void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S, &Pc};
-  return tc::launch_pdl((const void*)gemv_ring_kernel<MX>, dim3(p.grid, num_problems), dim3(kRingThreads), p.smem,
+  return tc::launch_pdl((const void*)gemv_ring_kernel<MX, GROUPED>, dim3(p.grid, num_problems), dim3(kRingThreads), p.smem,
                         stream, args);
 }
 
@@ -749,19 +750,19 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
 
 namespace {
 
-template <bool MX>
+template <bool MX, bool GROUPED>
 cudaError_t launch_any(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
                        int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream, const Problems& P,
                        int num_problems) {
   RingPlan plan;
   if (ring_plan(N, K, sms, MX, num_problems, plan)) {
     bool encoded = false;
-    const cudaError_t e = launch_ring<MX>(x, q, s, g, y, N, K, stream, plan, P, num_problems, &encoded);
+    const cudaError_t e = launch_ring<MX, GROUPED>(x, q, s, g, y, N, K, stream, plan, P, num_problems, &encoded);
     if (encoded || e != cudaSuccess) return e;
   }
   if (MX || K % 32 == 0)
-    return launch<8, 16, 2, MX>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
-  return launch<8, 8, 2, false>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
+    return launch<8, 16, 2, MX, GROUPED>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
+  return launch<8, 8, 2, false, GROUPED>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
 }
 
 const Problems kSingle = {nullptr, nullptr, 1, 1, 0, 0};
@@ -770,12 +771,12 @@ const Problems kSingle = {nullptr, nullptr, 1, 1, 0, 0};
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                         uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  return launch_any<false>(x, q, s, g, y, N, K, sms, static_weights, stream, kSingle, 1);
+  return launch_any<false, false>(x, q, s, g, y, N, K, sms, static_weights, stream, kSingle, 1);
 }
 
 cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
                            int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  return launch_any<true>(x, q, s, nullptr, y, N, K, sms, static_weights, stream, kSingle, 1);
+  return launch_any<true, false>(x, q, s, nullptr, y, N, K, sms, static_weights, stream, kSingle, 1);
 }
 
 cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
@@ -783,7 +784,7 @@ cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q
                                 int64_t ldy, int64_t P, int64_t E, int64_t T, int64_t N, int64_t K, int sms,
                                 cudaStream_t stream) {
   const Problems pr = {expert_ids, token_ids, (int)E, (int)T, ldx, ldy};
-  return launch_any<false>(X, q, s, g, Y, N, K, sms, false, stream, pr, (int)P);
+  return launch_any<false, true>(X, q, s, g, Y, N, K, sms, false, stream, pr, (int)P);
 }
 
 cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count) {
