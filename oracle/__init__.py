@@ -267,3 +267,44 @@ def linear_grouped(X, q: np.ndarray, s: np.ndarray, g: np.ndarray, expert_ids, t
         yp, bp = linear(xb[t:t + 1], q[e], s[e], g[e])
         y[p], bound[p] = yp[0], bp[0]
     return y, bound
+
+
+# ------------------------------------------- MXFP4 scales as NVFP4 scales
+
+def _e4m3_byte_of_pow2(j: int) -> int:
+    """E4M3 code of 2^j for j in [-9, 8] (subnormals below 2^-6)."""
+    assert -9 <= j <= 8
+    return (j + 7) << 3 if j >= -6 else 1 << (j + 9)
+
+
+def mx_to_nvfp4(q: np.ndarray, s_mx: np.ndarray):
+    """The same weights in NVFP4 form: the codes stay, each UE8M0 block scale
+    2^k (32 elements) becomes the E4M3 scale 2^(k - G) of its two 16-element
+    halves, with the tensor scale g = 2^G, G = (largest k of a block with a
+    non-zero code) - 8.  Exact when every such block has k - G >= -9 (E4M3
+    holds the powers 2^-9 .. 2^8); blocks whose codes are all zero get scale 0.
+    Returns (s_nv [N, K/16], g, number of non-zero blocks outside the window,
+    which get scale 0)."""
+    q = np.ascontiguousarray(q, np.uint8)
+    s_mx = np.ascontiguousarray(s_mx, np.uint8)
+    N, nb = s_mx.shape
+    mags = np.stack([q & 7, (q >> 4) & 7], axis=-1).reshape(N, nb, 32)
+    nonzero = mags.any(axis=2)
+    k = s_mx.astype(np.int64) - 127
+    if nonzero.any():
+        G = int(k[nonzero].max()) - 8
+    else:
+        G = 0
+    s_nv = np.zeros((N, nb), np.uint8)
+    bad = 0
+    for n in range(N):
+        for b in range(nb):
+            if not nonzero[n, b]:
+                continue
+            j = int(k[n, b]) - G
+            if j < -9:
+                bad += 1
+                continue
+            s_nv[n, b] = _e4m3_byte_of_pow2(j)
+    g = np.float32(np.ldexp(1.0, G))
+    return np.repeat(s_nv, 2, axis=1), g, bad
