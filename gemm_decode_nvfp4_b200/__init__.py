@@ -22,7 +22,7 @@ __all__ = [
     "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
     "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
-    "mx_quantize", "mx_quantize_new", "mx_gemv", "gemv_grouped",
+    "mx_quantize", "mx_quantize_new", "mx_gemv", "gemv_grouped", "mx_to_nvfp4",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -50,13 +50,14 @@ lib.nvfp4_gemm_workspace_size.argtypes = [_i64, _i64, _i64]
 lib.nvfp4_gemv_grouped.argtypes = [_p, _i64, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64,
                                    ctypes.c_uint32, _p]
 lib.mxfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p]
+lib.mxfp4_to_nvfp4_scales.argtypes = [_p, _p, _i64, _i64, _p, _p, _p]
 lib.mxfp4_gemv.argtypes = [_p, _p, _p, _p, _i64, _i64, _p]
 lib.mxfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
 for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
            lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors, lib.mxfp4_quantize, lib.mxfp4_gemv,
-           lib.mxfp4_gemv_ex, lib.nvfp4_gemv_grouped):
+           lib.mxfp4_gemv_ex, lib.nvfp4_gemv_grouped, lib.mxfp4_to_nvfp4_scales):
     _f.restype = ctypes.c_int
 
 
@@ -313,3 +314,19 @@ def gemv_grouped(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Ten
     _check("nvfp4_gemv_grouped", lib.nvfp4_gemv_grouped(
         _ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(expert_ids), _ptr(token_ids), _ptr(Y), Y.stride(0),
         P, E, T, N, K, 0, _stream(stream)))
+
+
+def mx_to_nvfp4(q: torch.Tensor, s_mx: torch.Tensor, stream=None):
+    """MXFP4 scales s_mx [N, K/32] restated as NVFP4 scales [N, K/16] and a
+    power-of-two tensor scale g [1] (exact within 17 binades; see
+    include/mxfp4.h), so that (q, s_nv, g) runs on gemv/gemm."""
+    _need(q, torch.uint8, "q", 2)
+    _need(s_mx, torch.uint8, "s_mx", 2)
+    N, K = q.shape[0], q.shape[1] * 2
+    if not q.is_contiguous() or not s_mx.is_contiguous() or s_mx.shape != (N, K // 32):
+        raise ValueError("q/s_mx must be contiguous [N, K/2] / [N, K/32]")
+    s_nv = torch.empty((N, K // 16), dtype=torch.uint8, device=q.device)
+    g = torch.empty((1,), dtype=torch.float32, device=q.device)
+    _check("mxfp4_to_nvfp4_scales", lib.mxfp4_to_nvfp4_scales(_ptr(q), _ptr(s_mx), N, K, _ptr(s_nv), _ptr(g),
+                                                               _stream(stream)))
+    return s_nv, g

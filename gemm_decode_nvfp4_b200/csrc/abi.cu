@@ -240,6 +240,25 @@ nvfp4_status mxfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "mxfp4 quantize launch");
 }
 
+nvfp4_status mxfp4_to_nvfp4_scales(const uint8_t* q, const uint8_t* s_mx, int64_t N, int64_t K, uint8_t* s_nv,
+                                   float* g_out, nvfp4_stream_t stream) {
+  if (K <= 0 || K % 32 != 0) return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 32", (long long)K);
+  if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
+  if (N == 0) return NVFP4_OK;
+  if (!q || !s_mx || !s_nv || !g_out) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(q) || !aligned16(s_mx) || !aligned16(s_nv) || !aligned4(g_out))
+    return fail(NVFP4_ERR_ALIGNMENT, "q, s_mx, s_nv must be 16-byte and g_out 4-byte aligned");
+  const size_t qb = (size_t)(N * K / 2), mb = (size_t)(N * K / 32), nb = (size_t)(N * K / 16);
+  if (overlaps(s_nv, nb, q, qb) || overlaps(s_nv, nb, s_mx, mb) || overlaps(g_out, 4, q, qb) ||
+      overlaps(g_out, 4, s_mx, mb) || overlaps(g_out, 4, s_nv, nb))
+    return fail(NVFP4_ERR_INVALID_ARG, "s_nv and g_out must not overlap the inputs or each other");
+  int sms = 0;
+  nvfp4_status st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_mx_to_nvfp4(q, s_mx, N, K, s_nv, g_out, (cudaStream_t)stream, sms);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "mxfp4 scale conversion launch");
+}
+
 nvfp4_status mxfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
                         int64_t K, nvfp4_stream_t stream) {
   return mxfp4_gemv_ex(x, q, s, y, N, K, 0u, stream);
@@ -349,12 +368,16 @@ nvfp4_status nvfp4_check_device_errors(void) {
   cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_small_timeouts(&k);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_timeouts(&v);
-  unsigned int bad = 0;
+  unsigned int bad = 0, window = 0;
   if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_bad_ids(&bad);
+  if (e == cudaSuccess) e = nvfp4::read_and_clear_mx_out_of_window(&window);
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error counter");
   if (n || k || v)
     return fail(NVFP4_ERR_TIMEOUT, "%u GEMM, %u small-M GEMM and %u GEMV CTA(s) gave up on a pipeline wait", n, k, v);
   if (bad) return fail(NVFP4_ERR_INVALID_ARG, "%u grouped GEMV problem(s) had an out-of-range expert or token id", bad);
+  if (window)
+    return fail(NVFP4_ERR_INVALID_ARG, "%u MXFP4 block(s) could not be restated as NVFP4 scales (more than 17 binades "
+                "below the largest, or NaN)", window);
   return NVFP4_OK;
 }
 

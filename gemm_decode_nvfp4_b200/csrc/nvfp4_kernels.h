@@ -35,6 +35,12 @@ cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q
                                 cudaStream_t stream);
 // Problems of grouped GEMVs whose ids were out of range since the last read.
 cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count);
+// MXFP4 scales restated as NVFP4 scales s_nv [N, K/16] and a power-of-two
+// tensor scale g (quantize.cu); non-zero blocks outside the E4M3 window are
+// counted (read_and_clear_mx_out_of_window).
+cudaError_t launch_mx_to_nvfp4(const uint8_t* q, const uint8_t* s_mx, int64_t N, int64_t K, uint8_t* s_nv,
+                               float* g, cudaStream_t stream, int sms);
+cudaError_t read_and_clear_mx_out_of_window(unsigned int* count);
 // MXFP4 round-to-nearest quantizer (quantize.cu); K a multiple of 32.
 cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, uint8_t* q, uint8_t* s,
                                cudaStream_t stream, int sms);

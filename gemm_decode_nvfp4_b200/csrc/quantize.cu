@@ -239,6 +239,64 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
   }
 }
 
+// ----------------------------------------------- MXFP4 scales as NVFP4 scales
+//
+// The two formats share the nibble layout, so MXFP4 weights run on the NVFP4
+// GEMMs once their scales are restated: with g = 2^G, a UE8M0 block scale 2^k
+// is the E4M3 scale 2^(k - G) of both 16-element halves of its 32-block (E4M3
+// holds the powers 2^-9 .. 2^8).  G = (largest k of a block with a non-zero
+// code) - 8, found by a max-reduction into the g slot itself (as an int,
+// starting from the byte pattern 0x80808080), so no scratch memory is needed.
+
+// Blocks with the NaN scale byte 255, and non-zero blocks whose scale fell
+// outside the E4M3 window.
+__device__ unsigned int g_mx_out_of_window = 0;
+
+constexpr int kNoBlock = (int)0x80808080;  // the reduction's start value: no non-zero block yet
+
+__device__ __forceinline__ bool mx_block_nonzero(const uint8_t* q, int64_t b) {
+  const uint4 w = *reinterpret_cast<const uint4*>(q + 16 * b);
+  return ((w.x | w.y | w.z | w.w) & 0x77777777u) != 0u;  // any magnitude bits (codes 0x0 / 0x8 are zeros)
+}
+
+__global__ void __launch_bounds__(256) mx_kmax_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
+                                                      int64_t nblocks, int* __restrict__ kmax) {
+  int m = kNoBlock;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblocks; b += stride)
+    if (s[b] != 255u && mx_block_nonzero(q, b)) m = max(m, (int)s[b] - 127);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m != kNoBlock) atomicMax(kmax, m);
+}
+
+__device__ __forceinline__ int mx_tensor_exponent(int kmax) { return kmax == kNoBlock ? 0 : kmax - 8; }
+
+__global__ void __launch_bounds__(256) mx_to_nv_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
+                                                       int64_t nblocks, const int* __restrict__ kmax,
+                                                       uint8_t* __restrict__ s_nv) {
+  const int G = mx_tensor_exponent(*kmax);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+    uint32_t byte = 0;
+    if (s[b] == 255u) {  // NaN scale: no finite NVFP4 scale holds it
+      atomicAdd(&g_mx_out_of_window, 1u);
+    } else if (mx_block_nonzero(q, b)) {
+      const int j = (int)s[b] - 127 - G;
+      if (j < -9)
+        atomicAdd(&g_mx_out_of_window, 1u);
+      else
+        byte = j >= -6 ? (uint32_t)(j + 7) << 3 : 1u << (j + 9);  // 2^j in E4M3 (subnormal below 2^-6)
+    }
+    *reinterpret_cast<uint16_t*>(s_nv + 2 * b) = (uint16_t)(byte | (byte << 8));
+  }
+}
+
+__global__ void mx_g_kernel(float* g) {  // the reduced exponent in the g slot -> g = 2^G
+  const int G = mx_tensor_exponent(*reinterpret_cast<const int*>(g));
+  *g = G >= -126 ? __uint_as_float((uint32_t)(G + 127) << 23) : __uint_as_float(1u << (G + 149));
+}
+
 __global__ void finalize_scale_kernel(float* amax_then_g) {
   *amax_then_g = __fdiv_rn(*amax_then_g, 2688.0f);
 }
@@ -271,6 +329,25 @@ cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t 
   const int grid = grid_for(N * (K / 32), sms);
   mx_quantize_kernel<<<grid, 256, 0, stream>>>(w, N, K, ldw, q, s);
   return cudaGetLastError();
+}
+
+cudaError_t launch_mx_to_nvfp4(const uint8_t* q, const uint8_t* s_mx, int64_t N, int64_t K, uint8_t* s_nv,
+                               float* g, cudaStream_t stream, int sms) {
+  const int64_t nblocks = N * (K / 32);
+  cudaError_t e = cudaMemsetAsync(g, 0x80, sizeof(float), stream);  // kNoBlock
+  if (e != cudaSuccess) return e;
+  const int grid = grid_for(nblocks, sms);
+  mx_kmax_kernel<<<grid, 256, 0, stream>>>(q, s_mx, nblocks, reinterpret_cast<int*>(g));
+  mx_to_nv_kernel<<<grid, 256, 0, stream>>>(q, s_mx, nblocks, reinterpret_cast<const int*>(g), s_nv);
+  mx_g_kernel<<<1, 1, 0, stream>>>(g);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_mx_out_of_window(unsigned int* count) {
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_mx_out_of_window, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_mx_out_of_window, &zero, sizeof(unsigned int));
 }
 
 cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream) {

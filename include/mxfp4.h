@@ -55,6 +55,23 @@ NVFP4_API nvfp4_status mxfp4_gemv(const uint16_t* x, const uint8_t* q, const uin
 NVFP4_API nvfp4_status mxfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y,
                                      int64_t N, int64_t K, uint32_t flags, nvfp4_stream_t stream);
 
+/*
+ * MXFP4 weights on the NVFP4 kernels (nvfp4_gemm, nvfp4_gemv, ...): the codes q
+ * are shared, and the scales are restated once (weights are static) as NVFP4
+ * scales s_nv [N, K/16] with a power-of-two tensor scale *g_out:
+ *   G = (largest k = s_mx - 127 over blocks with a non-zero code) - 8,
+ *   s_nv of both 16-element halves of a 32-block = E4M3(2^(k - G)), g = 2^G,
+ * which reproduces the MXFP4 weights exactly when every non-zero block lies
+ * within 17 binades of the largest (E4M3 holds 2^-9 .. 2^8).  Blocks whose
+ * codes are all zero get scale 0.  Blocks with the NaN scale byte 255 (which
+ * take no part in G) and non-zero blocks outside the window get scale 0 and
+ * are counted: nvfp4_check_device_errors then returns NVFP4_ERR_INVALID_ARG.  q, s_mx, s_nv 16-byte aligned and
+ * contiguous; g_out 4-byte aligned (it also holds the reduction while the call
+ * runs).  N == 0 is a no-op.
+ */
+NVFP4_API nvfp4_status mxfp4_to_nvfp4_scales(const uint8_t* q, const uint8_t* s_mx, int64_t N, int64_t K,
+                                             uint8_t* s_nv, float* g_out, nvfp4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

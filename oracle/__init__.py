@@ -283,20 +283,23 @@ def mx_to_nvfp4(q: np.ndarray, s_mx: np.ndarray):
     halves, with the tensor scale g = 2^G, G = (largest k of a block with a
     non-zero code) - 8.  Exact when every such block has k - G >= -9 (E4M3
     holds the powers 2^-9 .. 2^8); blocks whose codes are all zero get scale 0.
-    Returns (s_nv [N, K/16], g, number of non-zero blocks outside the window,
+    A block with scale byte 255 decodes to NaN (e8m0_decode), which no finite
+    NVFP4 scale holds: it takes no part in G and is counted like a block
+    outside the window.  Returns (s_nv [N, K/16], g, number of counted blocks,
     which get scale 0)."""
     q = np.ascontiguousarray(q, np.uint8)
     s_mx = np.ascontiguousarray(s_mx, np.uint8)
     N, nb = s_mx.shape
     mags = np.stack([q & 7, (q >> 4) & 7], axis=-1).reshape(N, nb, 32)
-    nonzero = mags.any(axis=2)
+    nan_block = s_mx == 255
+    nonzero = mags.any(axis=2) & ~nan_block
     k = s_mx.astype(np.int64) - 127
     if nonzero.any():
         G = int(k[nonzero].max()) - 8
     else:
         G = 0
     s_nv = np.zeros((N, nb), np.uint8)
-    bad = 0
+    bad = int(nan_block.sum())
     for n in range(N):
         for b in range(nb):
             if not nonzero[n, b]:

@@ -47,3 +47,16 @@ def test_all_zero_tensor():
     s = np.full((3, 4), 200, np.uint8)
     s_nv, g, bad = oracle.mx_to_nvfp4(q, s)
     assert bad == 0 and g == 1.0 and not s_nv.any()
+
+
+def test_nan_scale_blocks_are_counted_and_ignored():
+    """Scale byte 255 is NaN in UE8M0 (library decode): such blocks, zero codes
+    or not, are counted and leave G to the finite blocks."""
+    q, s = _mx(4, 128, 3, 118, 124)
+    assert np.isnan(np.array([255], np.uint8).view(ml_dtypes.float8_e8m0fnu).astype(np.float64)[0])
+    s[1, 2] = 255
+    q[2, 0:16] = 0
+    s[2, 0] = 255
+    s_nv, g, bad = oracle.mx_to_nvfp4(q, s)
+    assert bad == 2 and not s_nv[1, 4:6].any() and not s_nv[2, 0:2].any()
+    assert g == np.float32(2.0 ** (int(s[s != 255].max()) - 127 - 8))
