@@ -311,3 +311,30 @@ def mx_to_nvfp4(q: np.ndarray, s_mx: np.ndarray):
             s_nv[n, b] = _e4m3_byte_of_pow2(j)
     g = np.float32(np.ldexp(1.0, G))
     return np.repeat(s_nv, 2, axis=1), g, bad
+
+
+def w4a4_linear(x, q: np.ndarray, s: np.ndarray, g, x_amax=None, rows=None, cols=None):
+    """W4A4 product (the pages' NVFP4 x NVFP4 prefill GEMM, imp
+    docs/quantization.md, dense-layer pipeline and the Modelopt row of the
+    tools table).  The pages give no activation rule; the reading taken is the
+    weights' own: X is quantized round-to-nearest to NVFP4 with the tensor
+    scale g_x = x_amax / 2688 (x_amax = max |X| when not given, as a calibrated
+    input scale would be), then y = X_deq . W_deq^T in fp64 with the bound
+    sum |x_deq w_deq|.
+
+    x is BF16 [M, K]; with rows/cols only those outputs are computed (1-D
+    results).  Returns (y, bound, (qx, sx, g_x))."""
+    xb = _bf16_bits(x)
+    if xb.ndim == 1:
+        xb = xb.reshape(1, -1)
+    g_x = tensor_scale(amax(xb) if x_amax is None else x_amax)
+    qx, sx, g_x = quantize(xb, g_x)
+    xd = dequantize(qx, sx, g_x)
+    if rows is None:
+        wd = dequantize(q, s, g)
+        return xd @ wd.T, np.abs(xd) @ np.abs(wd).T, (qx, sx, g_x)
+    ri = np.asarray(rows, np.int64)
+    ci = np.asarray(cols, np.int64)
+    wd = dequantize(np.asarray(q)[ci], np.asarray(s)[ci], g)
+    xr = xd[ri]
+    return (xr * wd).sum(axis=1), (np.abs(xr) * np.abs(wd)).sum(axis=1), (qx, sx, g_x)
