@@ -23,12 +23,15 @@ __all__ = [
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
     "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
     "mx_quantize", "mx_quantize_new", "mx_gemv", "gemv_grouped", "mx_to_nvfp4",
+    "GIVEN_AMAX", "w4a4_prepare_weights", "w4a4_quantize_x", "w4a4_gemm", "w4a4_linear",
+    "w4a4_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
 MX_HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "mxfp4.h")
+W4A4_HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "nvfp4_w4a4.h")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python gemm_decode_nvfp4_b200/build.py`")
@@ -51,13 +54,22 @@ lib.nvfp4_gemv_grouped.argtypes = [_p, _i64, _p, _p, _p, _p, _p, _p, _i64, _i64,
                                    ctypes.c_uint32, _p]
 lib.mxfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p]
 lib.mxfp4_to_nvfp4_scales.argtypes = [_p, _p, _i64, _i64, _p, _p, _p]
+lib.nvfp4_w4a4_weight_scales_bytes.argtypes, lib.nvfp4_w4a4_weight_scales_bytes.restype = [_i64, _i64], _sz
+lib.nvfp4_w4a4_x_scales_bytes.argtypes, lib.nvfp4_w4a4_x_scales_bytes.restype = [_i64, _i64], _sz
+lib.nvfp4_w4a4_workspace_size.argtypes, lib.nvfp4_w4a4_workspace_size.restype = [_i64, _i64], _sz
+lib.nvfp4_w4a4_prepare_weights.argtypes = [_p, _i64, _i64, _p, _p]
+lib.nvfp4_w4a4_quantize_x.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, ctypes.c_uint32, _p]
+lib.nvfp4_w4a4_gemm.argtypes = [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_uint32, _p]
+lib.nvfp4_w4a4_linear.argtypes = [_p, _i64, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, ctypes.c_uint32, _p]
 lib.mxfp4_gemv.argtypes = [_p, _p, _p, _p, _i64, _i64, _p]
 lib.mxfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
 for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
            lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors, lib.mxfp4_quantize, lib.mxfp4_gemv,
-           lib.mxfp4_gemv_ex, lib.nvfp4_gemv_grouped, lib.mxfp4_to_nvfp4_scales):
+           lib.mxfp4_gemv_ex, lib.nvfp4_gemv_grouped, lib.mxfp4_to_nvfp4_scales,
+           lib.nvfp4_w4a4_prepare_weights, lib.nvfp4_w4a4_quantize_x, lib.nvfp4_w4a4_gemm,
+           lib.nvfp4_w4a4_linear):
     _f.restype = ctypes.c_int
 
 
@@ -84,9 +96,9 @@ def version() -> int:
 
 
 def declared_symbols() -> list[str]:
-    """Names of the entry points include/nvfp4.h and include/mxfp4.h declare."""
+    """Names of the entry points include/nvfp4.h, mxfp4.h and nvfp4_w4a4.h declare."""
     names = []
-    for path in (HEADER_PATH, MX_HEADER_PATH):
+    for path in (HEADER_PATH, MX_HEADER_PATH, W4A4_HEADER_PATH):
         with open(path) as f:
             names += re.findall(r"NVFP4_API\s+[\w\s\*]+?\b((?:nvfp4|mxfp4)_\w+)\s*\(", f.read())
     return names
@@ -330,3 +342,72 @@ def mx_to_nvfp4(q: torch.Tensor, s_mx: torch.Tensor, stream=None):
     _check("mxfp4_to_nvfp4_scales", lib.mxfp4_to_nvfp4_scales(_ptr(q), _ptr(s_mx), N, K, _ptr(s_nv), _ptr(g),
                                                                _stream(stream)))
     return s_nv, g
+
+
+# ----------------------------------------------------------------------- W4A4
+# NVFP4 x NVFP4 prefill (include/nvfp4_w4a4.h): activations quantized by the
+# weights' rule, block-scaled FP4 tensor-core GEMM.
+
+GIVEN_AMAX = 2  # NVFP4_W4A4_GIVEN_AMAX
+
+
+def w4a4_prepare_weights(s: torch.Tensor, K: int, stream=None) -> torch.Tensor:
+    """Row-major weight scales [N, K/16] -> the tensor-core scale layout (u8)."""
+    _need(s, torch.uint8, "s", 2)
+    N = s.shape[0]
+    if not s.is_contiguous() or s.shape[1] * 16 != K:
+        raise ValueError("s must be contiguous [N, K/16]")
+    out = torch.empty((lib.nvfp4_w4a4_weight_scales_bytes(N, K),), dtype=torch.uint8, device=s.device)
+    _check("nvfp4_w4a4_prepare_weights", lib.nvfp4_w4a4_prepare_weights(_ptr(s), N, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def w4a4_quantize_x(X: torch.Tensor, x_amax: torch.Tensor, given_amax: bool = False, stream=None):
+    """X [M, K] -> (qx [M, K/2], sx in the tensor-core scale layout); x_amax [1]
+    receives max |X| unless given_amax."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(x_amax, torch.float32, "x_amax")
+    M, K = X.shape
+    if X.stride(1) != 1:
+        raise ValueError("X rows must be contiguous")
+    ldx = X.stride(0)
+    qx = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
+    sx = torch.empty((lib.nvfp4_w4a4_x_scales_bytes(M, K),), dtype=torch.uint8, device=X.device)
+    _check("nvfp4_w4a4_quantize_x", lib.nvfp4_w4a4_quantize_x(_ptr(X), ldx, M, K, _ptr(qx), _ptr(sx), _ptr(x_amax),
+                                                               GIVEN_AMAX if given_amax else 0, _stream(stream)))
+    return qx, sx
+
+
+def w4a4_gemm(qx, sx, x_amax, q, s_mma, g, Y, stream=None, static_weights: bool = False) -> None:
+    _need(Y, torch.bfloat16, "Y", 2)
+    M, N = Y.shape
+    K = q.shape[1] * 2
+    if qx.shape != (M, K // 2) or q.shape[0] != N:
+        raise ValueError(f"shape mismatch: qx {tuple(qx.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
+    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    _check("nvfp4_w4a4_gemm", lib.nvfp4_w4a4_gemm(_ptr(qx), _ptr(sx), _ptr(x_amax), _ptr(q), _ptr(s_mma), _ptr(g),
+                                                   _ptr(Y), Y.stride(0), M, N, K, flags, _stream(stream)))
+
+
+def w4a4_workspace_size(M: int, K: int) -> int:
+    return lib.nvfp4_w4a4_workspace_size(M, K)
+
+
+def w4a4_linear(X: torch.Tensor, q: torch.Tensor, s_mma: torch.Tensor, g: torch.Tensor, Y: torch.Tensor,
+                workspace: torch.Tensor, x_amax: torch.Tensor | None = None, stream=None,
+                static_weights: bool = False) -> None:
+    """Y [M, N] = W4A4 product of BF16 X [M, K] (quantized on the fly into the
+    workspace) and NVFP4 weights (q, s_mma from w4a4_prepare_weights, g)."""
+    _need(X, torch.bfloat16, "X", 2)
+    _need(Y, torch.bfloat16, "Y", 2)
+    _need(workspace, torch.uint8, "workspace")
+    M, K = X.shape
+    N = q.shape[0]
+    if q.shape[1] * 2 != K or Y.shape != (M, N):
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
+    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    if X.stride(1) != 1:
+        raise ValueError("X rows must be contiguous")
+    _check("nvfp4_w4a4_linear", lib.nvfp4_w4a4_linear(_ptr(X), X.stride(0), _ptr(x_amax), _ptr(q), _ptr(s_mma),
+                                                       _ptr(g), _ptr(Y), Y.stride(0), M, N, K, _ptr(workspace),
+                                                       workspace.numel(), flags, _stream(stream)))

@@ -8,6 +8,7 @@
 #include "mxfp4.h"
 #include "nvfp4.h"
 #include "nvfp4_kernels.h"
+#include "nvfp4_w4a4.h"
 
 namespace {
 
@@ -363,9 +364,142 @@ nvfp4_status nvfp4_gemm_ex(const uint16_t* X, int64_t ldx, const uint8_t* q, con
   return NVFP4_OK;
 }
 
+// ------------------------------------------------------------------- W4A4
+
+namespace {
+
+size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+nvfp4_status check_w4a4_shape(int64_t M, int64_t N, int64_t K) {
+  if (K <= 0 || K % 256 != 0 || K > ((int64_t)1 << 24))
+    return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 256, at most 2^24", (long long)K);
+  if (M < 0 || N < 0) return fail(NVFP4_ERR_SHAPE, "negative size M=%lld N=%lld", (long long)M, (long long)N);
+  if (M > ((int64_t)1 << 24) || N > ((int64_t)1 << 31) - 128)
+    return fail(NVFP4_ERR_SHAPE, "M=%lld or N=%lld too large", (long long)M, (long long)N);
+  return NVFP4_OK;
+}
+
+}  // namespace
+
+size_t nvfp4_w4a4_weight_scales_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0 || K % 256) return 0;
+  return round_up((size_t)N, 128) * (size_t)(K / 16);
+}
+
+size_t nvfp4_w4a4_x_scales_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0 || K % 256) return 0;
+  return round_up((size_t)M, 256) * (size_t)(K / 16);
+}
+
+size_t nvfp4_w4a4_workspace_size(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0 || K % 256) return 0;
+  return round_up((size_t)(M * K / 2), 16) + nvfp4_w4a4_x_scales_bytes(M, K) + 16;
+}
+
+nvfp4_status nvfp4_w4a4_prepare_weights(const uint8_t* s, int64_t N, int64_t K, uint8_t* s_mma,
+                                        nvfp4_stream_t stream) {
+  nvfp4_status st = check_w4a4_shape(1, N, K);
+  if (st != NVFP4_OK) return st;
+  if (N == 0) return NVFP4_OK;
+  if (!s || !s_mma) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(s) || !aligned16(s_mma)) return fail(NVFP4_ERR_ALIGNMENT, "s and s_mma must be 16-byte aligned");
+  if (overlaps(s, (size_t)(N * K / 16), s_mma, nvfp4_w4a4_weight_scales_bytes(N, K)))
+    return fail(NVFP4_ERR_INVALID_ARG, "s_mma must not overlap s");
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_scales_to_mma(s, N, K, s_mma, (cudaStream_t)stream, sms);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "scale rearrangement launch");
+}
+
+nvfp4_status nvfp4_w4a4_quantize_x(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, uint8_t* qx, uint8_t* sx,
+                                   float* x_amax, uint32_t flags, nvfp4_stream_t stream) {
+  if (flags & ~NVFP4_W4A4_GIVEN_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  nvfp4_status st = check_w4a4_shape(M, 1, K);
+  if (st != NVFP4_OK) return st;
+  if (M == 0) return NVFP4_OK;
+  if (!X || !qx || !sx || !x_amax) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (ldx < K) return fail(NVFP4_ERR_INVALID_ARG, "ldx=%lld < K=%lld", (long long)ldx, (long long)K);
+  if (!aligned16(X) || !aligned16(qx) || !aligned16(sx) || ldx % 8 || !aligned4(x_amax))
+    return fail(NVFP4_ERR_ALIGNMENT, "X, qx, sx must be 16-byte aligned, ldx a multiple of 8, x_amax 4-byte aligned");
+  const size_t xb = (size_t)((M - 1) * ldx + K) * 2, qb = (size_t)(M * K / 2), sb = nvfp4_w4a4_x_scales_bytes(M, K);
+  if (overlaps(X, xb, qx, qb) || overlaps(X, xb, sx, sb) || overlaps(qx, qb, sx, sb) || overlaps(x_amax, 4, X, xb) ||
+      overlaps(x_amax, 4, qx, qb) || overlaps(x_amax, 4, sx, sb))
+    return fail(NVFP4_ERR_INVALID_ARG, "X, qx, sx and x_amax must not overlap");
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (!(flags & NVFP4_W4A4_GIVEN_AMAX)) {
+    e = cudaMemsetAsync(x_amax, 0, sizeof(float), cs);
+    if (e == cudaSuccess) e = nvfp4::launch_amax(X, M, K, ldx, x_amax, cs, sms);
+    if (e != cudaSuccess) return cuda_fail(e, "activation amax launch");
+  }
+  e = nvfp4::launch_quantize_x_mma(X, ldx, M, K, x_amax, qx, sx, cs, sms);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "activation quantize launch");
+}
+
+nvfp4_status nvfp4_w4a4_gemm(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
+                             const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                             int64_t K, uint32_t flags, nvfp4_stream_t stream) {
+  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  nvfp4_status st = check_w4a4_shape(M, N, K);
+  if (st != NVFP4_OK) return st;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (!qx || !sx || !x_amax || !q || !s_mma || !g || !Y) return fail(NVFP4_ERR_INVALID_ARG, "null pointer");
+  if (ldy < N) return fail(NVFP4_ERR_INVALID_ARG, "ldy=%lld < N=%lld", (long long)ldy, (long long)N);
+  if (!aligned16(qx) || !aligned16(sx) || !aligned16(q) || !aligned16(s_mma))
+    return fail(NVFP4_ERR_ALIGNMENT, "qx, sx, q and s_mma must be 16-byte aligned");
+  if (!aligned4(x_amax) || !aligned4(g) || !aligned2(Y))
+    return fail(NVFP4_ERR_ALIGNMENT, "x_amax and g must be 4-byte aligned, Y 2-byte aligned");
+  const size_t yb = (size_t)((M - 1) * ldy + N) * 2;
+  if (overlaps(Y, yb, qx, (size_t)(M * K / 2)) || overlaps(Y, yb, sx, nvfp4_w4a4_x_scales_bytes(M, K)) ||
+      overlaps(Y, yb, q, (size_t)(N * K / 2)) || overlaps(Y, yb, s_mma, nvfp4_w4a4_weight_scales_bytes(N, K)) ||
+      overlaps(Y, yb, g, 4) || overlaps(Y, yb, x_amax, 4))
+    return fail(NVFP4_ERR_INVALID_ARG, "Y must not overlap an input");
+  int sms = 0;
+  st = check_device(&sms);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_gemm_w4a4(qx, sx, x_amax, q, s_mma, g, Y, ldy, M, N, K,
+                                          (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0, (cudaStream_t)stream);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "W4A4 GEMM launch");
+}
+
+nvfp4_status nvfp4_w4a4_linear(const uint16_t* X, int64_t ldx, const float* x_amax, const uint8_t* q,
+                               const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                               int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
+                               nvfp4_stream_t stream) {
+  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  nvfp4_status st = check_w4a4_shape(M, N, K);
+  if (st != NVFP4_OK) return st;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  const size_t need = nvfp4_w4a4_workspace_size(M, K);
+  if (!workspace || workspace_bytes < need)
+    return fail(NVFP4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+  if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  if (X && ldx >= K) {
+    const size_t xb = (size_t)((M - 1) * ldx + K) * 2, yb = ldy >= N ? (size_t)((M - 1) * ldy + N) * 2 : 0;
+    if (overlaps(workspace, need, X, xb) || overlaps(workspace, need, Y, yb) ||
+        overlaps(workspace, need, q, (size_t)(N * K / 2)) ||
+        overlaps(workspace, need, s_mma, nvfp4_w4a4_weight_scales_bytes(N, K)) || overlaps(workspace, need, g, 4) ||
+        (x_amax && overlaps(workspace, need, x_amax, 4)))
+      return fail(NVFP4_ERR_INVALID_ARG, "workspace must not overlap the other buffers");
+  }
+  uint8_t* qx = static_cast<uint8_t*>(workspace);
+  uint8_t* sx = qx + round_up((size_t)(M * K / 2), 16);
+  // the dynamic amax goes to the workspace's last slot; a given one is only read
+  float* amax = x_amax ? const_cast<float*>(x_amax) : reinterpret_cast<float*>(sx + nvfp4_w4a4_x_scales_bytes(M, K));
+  st = nvfp4_w4a4_quantize_x(X, ldx, M, K, qx, sx, amax, x_amax ? NVFP4_W4A4_GIVEN_AMAX : 0u, stream);
+  if (st != NVFP4_OK) return st;
+  return nvfp4_w4a4_gemm(qx, sx, amax, q, s_mma, g, Y, ldy, M, N, K, flags, stream);
+}
+
 nvfp4_status nvfp4_check_device_errors(void) {
-  unsigned int n = 0, k = 0, v = 0;
+  unsigned int n = 0, k = 0, v = 0, w = 0;
   cudaError_t e = nvfp4::read_and_clear_gemm_timeouts(&n);
+  if (e == cudaSuccess) e = nvfp4::read_and_clear_w4a4_timeouts(&w);
+  n += w;
   if (e == cudaSuccess) e = nvfp4::read_and_clear_small_timeouts(&k);
   if (e == cudaSuccess) e = nvfp4::read_and_clear_gemv_timeouts(&v);
   unsigned int bad = 0, window = 0;

@@ -1,0 +1,328 @@
+// gemm_w4a4.cu -- NVFP4 x NVFP4 (W4A4) prefill GEMM on the sm_100a block-scaled
+// FP4 tensor cores (tcgen05.mma kind::mxf4nvf4).
+//
+// The pages' prefill runs weights and activations both in NVFP4 ("CUTLASS
+// NVFP4 GEMM" of the dense-layer pipeline, imp docs/quantization.md; the
+// Modelopt row's "NVFP4 x NVFP4 prefill"), with the weight micro-scales
+// rearranged once into the tensor core's scale-factor layout ("Phase 3b").
+// Here:
+//   Y[m, n] = bf16(g * g_x * sum_k (sw[n, k/16] qw[n, k]) (sx[m, k/16] qx[m, k]))
+// with g_x = x_amax / 2688 and X quantized by the weights' rule
+// (quantize_x_mma_kernel).  Every product of two E2M1 codes and two E4M3
+// scales is exact in fp32; the tensor core accumulates in fp32.
+//
+// Scale-factor layout (weights and activations alike): one 512-byte atom per
+// 128 rows and 64 k; row r, 16-block j of the step at byte
+// (r % 32) * 16 + (r / 32) * 4 + j.  One tcgen05.cp (32 rows x 16 bytes,
+// replicated into the four lane quarters) moves an atom into 4 TMEM columns,
+// where the MMA reads row r at lane r % 32, column r / 32, byte j.
+//
+// Tile: 128 weight rows (MMA M, operand A) x 256 tokens (MMA N, operand B),
+// 256 k per pipeline stage (one 128-byte swizzled row of packed codes, four
+// MMAs of K = 64):
+//   - warp 0, one thread: TMA loads of the weight codes [128, 128 B] and the
+//     token codes [256, 128 B] (out-of-range rows read as zero) and bulk
+//     copies of the stage's scale atoms (2 KB of weights, 2 x 2 KB of tokens);
+//   - warp 1, one thread: per MMA, three tcgen05.cp of its scale atoms into
+//     the stage's own TMEM columns, then the MMA into the [128 x 256] fp32
+//     accumulator; each stage is committed to its "empty" barrier;
+//   - warps 2..5: the epilogue, TMEM -> g * g_x -> BF16 Y through shared memory.
+// A stage's TMEM scale columns are rewritten only after the MMAs that read
+// them have completed (the stage's empty barrier), and tcgen05.cp is ordered
+// before the MMAs its thread issues after it.  Every wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "nvfp4_device.cuh"
+#include "nvfp4_kernels.h"
+#include "sm100_ptx.cuh"
+#include "tc_host.h"
+
+namespace nvfp4 {
+
+// CTAs of the W4A4 GEMM whose pipeline wait ran past its time limit.
+__device__ unsigned int g_w4a4_wait_timeouts = 0;
+
+namespace {
+
+constexpr int kBM = 128;                      // weight rows per tile (MMA M)
+constexpr int kBN = 256;                      // tokens per tile (MMA N)
+constexpr int kStageK = 256;                  // k per pipeline stage
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * 128;            // packed weight codes of a stage
+constexpr int kBBytes = kBN * 128;            // packed token codes of a stage
+constexpr int kSFABytes = 4 * 512;            // weight scale atoms (4 MMAs)
+constexpr int kSFBBytes = 2 * 4 * 512;        // token scale atoms (2 x 128 tokens, 4 MMAs)
+constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+constexpr int kThreads = 6 * 32;
+constexpr int kEpiWarp0 = 2;
+constexpr uint32_t kTmemCols = 512;           // 256 accumulator + 4 stages x 4 MMAs x 12 scale columns
+constexpr uint32_t kSfCol0 = 256;
+constexpr uint32_t kSfColsPerMma = 12;        // 4 weight + 8 token columns
+constexpr uint32_t kIdesc = ptx::idesc_nvf4(kBM, kBN);
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle)");
+static_assert(kSfCol0 + kStages * 4 * kSfColsPerMma <= kTmemCols, "TMEM columns");
+
+struct Bars {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tmem_full;
+  uint32_t tmem_addr;
+  volatile int err;
+};
+
+constexpr int kSmemBytes = kStages * kStageBytes + (int)sizeof(Bars) + 1024;
+
+__device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Bars* bars) {
+  if (bars->err) return false;
+  if (ptx::mbar_wait(bar, parity, kWaitLimitNs)) return true;
+  if (!bars->err) {
+    bars->err = 1;
+    atomicAdd(&g_w4a4_wait_timeouts, 1u);
+  }
+  return false;
+}
+
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Rows of the weight scale rearrangement: thread t writes the 16 bytes of
+// atom row r0 for (tile, step): the four scale words of rows
+// tile*128 + 32*i + r0, i = 0..3 (zero beyond N).
+__global__ void __launch_bounds__(256) scales_to_mma_kernel(const uint8_t* __restrict__ s, int64_t N, int64_t K,
+                                                            uint8_t* __restrict__ s_mma) {
+  const int64_t steps = K / 64, tiles = (N + 127) / 128;
+  const int64_t total = tiles * steps * 32;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
+    const int64_t r0 = t % 32, atom = t / 32;  // atom = tile * steps + step
+    const int64_t tile = atom / steps, step = atom - tile * steps;
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t row = tile * 128 + 32 * i + r0;
+      w[i] = row < N ? *reinterpret_cast<const uint32_t*>(s + row * (K / 16) + step * 4) : 0u;
+    }
+    *reinterpret_cast<uint4*>(s_mma + atom * 512 + r0 * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                     const uint8_t* __restrict__ s_mma, const uint8_t* __restrict__ sx,
+                     const float* __restrict__ g, const float* __restrict__ x_amax, uint16_t* __restrict__ Y,
+                     int64_t ldy, int M, int N, int K, int static_weights) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  auto a_tile = [&](int st) { return smem + st * kStageBytes; };
+  auto b_tile = [&](int st) { return smem + st * kStageBytes + kABytes; };
+  auto sfa = [&](int st) { return smem + st * kStageBytes + kABytes + kBBytes; };
+  auto sfb = [&](int st) { return smem + st * kStageBytes + kABytes + kBBytes + kSFABytes; };
+  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nt = blockIdx.x, mt = blockIdx.y;
+  const int n0 = nt * kBM, m0 = mt * kBN;
+  const int steps64 = K / 64;
+  const int num_ks = K / kStageK;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      ptx::mbar_init(&bars->full[st], 1);
+      ptx::mbar_init(&bars->empty[st], 1);
+    }
+    ptx::mbar_init(&bars->tmem_full, 1);
+    bars->err = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmap_w);
+    ptx::prefetch_tmap(&tmap_x);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem_addr, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_addr;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint8_t* sa_src = s_mma + (int64_t)nt * steps64 * 512;
+      const uint8_t* sb_src0 = sx + (int64_t)(2 * mt) * steps64 * 512;
+      const uint8_t* sb_src1 = sx + (int64_t)(2 * mt + 1) * steps64 * 512;
+      auto issue_w = [&](int ks) {
+        const int st = ks % kStages;
+        ptx::tma_load_2d(a_tile(st), &tmap_w, &bars->full[st], ks * 128, n0);
+        ptx::bulk_load(sfa(st), sa_src + ks * kSFABytes, kSFABytes, &bars->full[st]);
+      };
+      auto issue_x = [&](int ks) {
+        const int st = ks % kStages;
+        ptx::tma_load_2d(b_tile(st), &tmap_x, &bars->full[st], ks * 128, m0);
+        ptx::bulk_load(sfb(st), sb_src0 + ks * 2048, 2048, &bars->full[st]);
+        ptx::bulk_load(sfb(st) + 2048, sb_src1 + ks * 2048, 2048, &bars->full[st]);
+      };
+      // static weights: the first stages' weights stream before the producer
+      // of X has finished
+      const int first = num_ks < kStages ? num_ks : kStages;
+      for (int ks = 0; ks < first; ++ks) ptx::mbar_arrive_expect_tx(&bars->full[ks], kStageBytes);
+      if (static_weights)
+        for (int ks = 0; ks < first; ++ks) issue_w(ks);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int ks = 0; ks < first; ++ks) {
+        if (!static_weights) issue_w(ks);
+        issue_x(ks);
+      }
+      int next = first;
+      for (; next < num_ks; ++next) {
+        const int st = next % kStages;
+        if (!wait_or_fail(&bars->empty[st], ((next / kStages) - 1) & 1, bars)) break;
+        ptx::mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
+        issue_w(next);
+        issue_x(next);
+      }
+      if (bars->err) {
+        // let the copies already issued land before the CTA exits
+        for (int ks = next > kStages ? next - kStages : 0; ks < next; ++ks)
+          ptx::mbar_wait(&bars->full[ks % kStages], (ks / kStages) & 1, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      for (int ks = 0; ks < num_ks; ++ks) {
+        const int st = ks % kStages;
+        if (!wait_or_fail(&bars->full[st], (ks / kStages) & 1, bars)) break;
+        ptx::tc_fence_after();
+        const uint32_t a0 = ptx::smem_u32(a_tile(st)), b0 = ptx::smem_u32(b_tile(st));
+        const uint32_t fa = ptx::smem_u32(sfa(st)), fb = ptx::smem_u32(sfb(st));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma;
+          ptx::tmem_copy_sf(col, ptx::rows16_desc(fa + kk * 512));
+          ptx::tmem_copy_sf(col + 4, ptx::rows16_desc(fb + kk * 512));
+          ptx::tmem_copy_sf(col + 8, ptx::rows16_desc(fb + 2048 + kk * 512));
+          ptx::mma_nvf4(tmem, ptx::sw128_kmajor_desc(a0 + 32 * kk), ptx::sw128_kmajor_desc(b0 + 32 * kk), kIdesc,
+                        col, col + 4, (ks | kk) != 0);
+        }
+        ptx::mma_commit(&bars->empty[st]);
+      }
+      // arrives when every MMA above is done (also on the error path, so that
+      // TMEM is never freed under a running MMA)
+      ptx::mma_commit(&bars->tmem_full);
+      if (bars->err) ptx::mbar_wait(&bars->tmem_full, 0, kWaitLimitNs);
+    }
+  } else {
+    // ----------------------------------------------------------------- epilogue
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x_amax and Y
+    const bool acc_ready = __all_sync(0xFFFFFFFFu, wait_or_fail(&bars->tmem_full, 0, bars));
+    if (acc_ready) {
+      ptx::tc_fence_after();
+      const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. +31 = weight rows
+      const float scale = __fmul_rn(*g, __fdiv_rn(*x_amax, 2688.0f));
+      // each 32 x 32 block (weight rows of this quarter x tokens) goes through
+      // 2 KB of the idle stage-0 buffers so that Y is written as 64-byte runs
+      const uint32_t stage = ptx::smem_u32(a_tile(0)) + (uint32_t)(warp - kEpiWarp0) * 2048u;
+      const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBN && m0 + c0 < M; c0 += 32) {
+        uint32_t rr[32];
+        ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(rr[j]) * scale);
+          st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
+          const int m = m0 + c0 + j;
+          const int nb = n0 + 32 * quarter + 8 * piece;
+          if (m < M && nb < N) {
+            const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
+            uint16_t* dst = Y + (int64_t)m * ldy + nb;
+            if (vec_ok && nb + 8 <= N) {
+              *reinterpret_cast<uint4*>(dst) = v;
+            } else {
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+              for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+int grid_for(int64_t work_items, int sms) {
+  const int64_t blocks = (work_items + 255) / 256;
+  const int64_t cap = (int64_t)sms * 8;
+  return (int)(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
+}
+
+}  // namespace
+
+cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t* s_mma, cudaStream_t stream,
+                                 int sms) {
+  const int64_t total = (N + 127) / 128 * (K / 64) * 32;
+  scales_to_mma_kernel<<<grid_for(total, sms), 256, 0, stream>>>(s, N, K, s_mma);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
+                             const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                             int64_t K, bool static_weights, cudaStream_t stream) {
+  CUtensorMap tw, tx;
+  if (!tc::make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
+                        128u, (uint32_t)kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !tc::make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, (uint64_t)(K / 2), (uint64_t)M, (uint64_t)(K / 2),
+                        128u, (uint32_t)kBN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  static bool attr_set[64] = {};  // per device ordinal
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  int m = (int)M, n = (int)N, k = (int)K, sw = static_weights ? 1 : 0;
+  void* args[] = {&tw, &tx, (void*)&s_mma, (void*)&sx, (void*)&g, (void*)&x_amax, &Y, &ldy, &m, &n, &k, &sw};
+  dim3 grid((unsigned)((N + kBM - 1) / kBM), (unsigned)((M + kBN - 1) / kBN));
+  return tc::launch_pdl((const void*)gemm_w4a4_kernel, grid, dim3(kThreads), kSmemBytes, stream, args);
+}
+
+cudaError_t read_and_clear_w4a4_timeouts(unsigned int* count) {
+  cudaError_t e = cudaMemcpyFromSymbol(count, g_w4a4_wait_timeouts, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_w4a4_wait_timeouts, &zero, sizeof(unsigned int));
+}
+
+}  // namespace nvfp4

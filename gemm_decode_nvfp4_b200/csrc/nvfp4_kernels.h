@@ -35,6 +35,20 @@ cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q
                                 cudaStream_t stream);
 // Problems of grouped GEMVs whose ids were out of range since the last read.
 cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count);
+// W4A4 (quantize.cu, gemm_w4a4.cu): X quantized by the weights' rule with
+// g_x = *x_amax / 2688 into row-major codes qx [M, K/2] and scales sx in the
+// tensor core's scale-factor layout (512-byte atoms per 128 rows x 64 k,
+// rows padded with zero scales to a multiple of 256); the weight scales
+// rearranged once into the same layout (rows padded to a multiple of 128);
+// the block-scaled FP4 GEMM Y = bf16(g * g_x * sum sx sw qx qw).
+cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, const float* x_amax,
+                                  uint8_t* qx, uint8_t* sx, cudaStream_t stream, int sms);
+cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t* s_mma, cudaStream_t stream,
+                                 int sms);
+cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
+                             const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
+                             int64_t K, bool static_weights, cudaStream_t stream);
+cudaError_t read_and_clear_w4a4_timeouts(unsigned int* count);
 // MXFP4 scales restated as NVFP4 scales s_nv [N, K/16] and a power-of-two
 // tensor scale g (quantize.cu); non-zero blocks outside the E4M3 window are
 // counted (read_and_clear_mx_out_of_window).

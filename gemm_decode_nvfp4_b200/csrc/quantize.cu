@@ -239,6 +239,57 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
   }
 }
 
+// ------------------------------------------------- activations for W4A4 GEMMs
+//
+// X [M, K] quantized by the weights' rule with g_x = x_amax / 2688: codes
+// row-major [M, K/2] and the E4M3 scales in the tensor core's scale-factor
+// layout: for row m and 64-element step kk, the four scale bytes of its
+// 16-blocks form one 32-bit word at byte
+//   ((m / 128) * (K / 64) + kk) * 512 + (m % 32) * 16 + ((m % 128) / 32) * 4,
+// i.e. one 512-byte atom per 128 rows and 64 k.  Rows M .. Mpad-1 get zero
+// scales (Mpad = M rounded up to 256, the GEMM's token tile).
+__global__ void __launch_bounds__(256) quantize_x_mma_kernel(const uint16_t* __restrict__ X, int64_t ldx,
+                                                             int64_t M, int64_t K, int64_t Mpad,
+                                                             const float* __restrict__ x_amax,
+                                                             uint8_t* __restrict__ qx, uint8_t* __restrict__ sx) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float g = __fdiv_rn(*x_amax, 2688.0f);
+  const int64_t steps = K / 64;
+  const int64_t total = Mpad * steps;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
+    const int64_t m = t / steps, kk = t - m * steps;
+    uint32_t word = 0;
+    if (m < M) {
+      const uint4* src = reinterpret_cast<const uint4*>(X + m * ldx + kk * 64);
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = ld_stream_v4(src + i);
+      uint2 codes[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t wv[8] = {v[2 * b].x, v[2 * b].y, v[2 * b].z, v[2 * b].w,
+                                v[2 * b + 1].x, v[2 * b + 1].y, v[2 * b + 1].z, v[2 * b + 1].w};
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          f[2 * i] = bf16lo_to_float(wv[i]);
+          f[2 * i + 1] = bf16hi_to_float(wv[i]);
+        }
+        uint32_t sc;
+        quantize_block(f, g, sc, codes[b]);
+        word |= sc << (8 * b);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(qx + m * (K / 2) + kk * 32);
+      dst[0] = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+      dst[1] = make_uint4(codes[2].x, codes[2].y, codes[3].x, codes[3].y);
+    }
+    const int64_t r = m % 128;
+    *reinterpret_cast<uint32_t*>(sx + ((m / 128) * steps + kk) * 512 + (r % 32) * 16 + (r / 32) * 4) = word;
+  }
+}
+
 // ----------------------------------------------- MXFP4 scales as NVFP4 scales
 //
 // The two formats share the nibble layout, so MXFP4 weights run on the NVFP4
@@ -329,6 +380,25 @@ cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t 
   const int grid = grid_for(N * (K / 32), sms);
   mx_quantize_kernel<<<grid, 256, 0, stream>>>(w, N, K, ldw, q, s);
   return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, const float* x_amax,
+                                  uint8_t* qx, uint8_t* sx, cudaStream_t stream, int sms) {
+  const int64_t Mpad = (M + 255) / 256 * 256;
+  const int grid = grid_for(Mpad * (K / 64), sms);
+  const int64_t ldx_ = ldx, M_ = M, K_ = K;
+  void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&Mpad, (void*)&x_amax, (void*)&qx,
+                  (void*)&sx};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, (const void*)quantize_x_mma_kernel, args);
 }
 
 cudaError_t launch_mx_to_nvfp4(const uint8_t* q, const uint8_t* s_mx, int64_t N, int64_t K, uint8_t* s_nv,

@@ -154,6 +154,29 @@ __device__ __forceinline__ void mma_ts_f16(uint32_t d_tmem, uint32_t a_tmem, uin
       : "memory");
 }
 
+// D[tmem] (+)= (A[smem] * SFA) * (B[smem] * SFB)^T with packed E2M1 A and B
+// (two codes per byte, the even k in the low nibble, K = 64 per MMA), one
+// UE4M3 scale per 16 elements of each row (kind::mxf4nvf4, block16), fp32
+// accumulate.  sfa_tmem / sfb_tmem: column addresses of the scale factors in
+// tensor memory (see tmem_copy_sf).
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy 32 rows x 16 bytes of shared memory (row i at src + 16 i, 512 bytes)
+// into tensor-memory columns taddr .. taddr+3 of lanes 0..31, replicated into
+// each of the four 32-lane quarters: lane i % 32 receives row i, its bytes 4c
+// .. 4c+3 in column taddr + c.  Ordered before later tcgen05.mma of this thread.
+__device__ __forceinline__ void tmem_copy_sf(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
 // Arrive once on `bar` when all tcgen05.mma issued so far by this thread are done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -216,6 +239,27 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
   d |= (uint64_t)1u << 46;                               // descriptor version (sm_100)
   d |= (uint64_t)2u << 61;                               // layout: 128-byte swizzle
   return d;
+}
+
+// Shared-memory descriptor of a K-major tile without swizzle whose rows are
+// 16 contiguous bytes (8-row core matrices 128 bytes apart): the source of
+// tmem_copy_sf.
+__device__ __forceinline__ uint64_t rows16_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);          // start address
+  d |= (uint64_t)(128u >> 4) << 32;                      // stride byte offset: next 8 rows
+  d |= (uint64_t)1u << 46;                               // descriptor version (sm_100)
+  return d;                                              // layout 0: no swizzle
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with E2M1 A and B, UE4M3 scales
+// per 16 elements, both operands K-major, tile M x N, K = 64 per MMA, scale
+// factors at byte 0 of their tensor-memory columns.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7)                          // A format E2M1
+         | (1u << 10)                       // B format E2M1
+         | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | ((uint32_t)(M >> 4) << 24);      // M / 16 (bit 23 = 0: UE4M3 scales)
 }
 
 // Instruction descriptor of kind::f16 with BF16 A and B, fp32 accumulator,

@@ -112,3 +112,39 @@ def test_grouped_validation():
     assert f(A, 64, A, A, A, A + 2, A, A + 8192, 16, 4, 4, 1, 16, 64, 0, None) == ALIGN
     assert f(A, 64, A + 8192, A + 16384, A + 24576, A + 32768, A + 32800, A, 16, 4, 4, 1, 16, 64, 0, None) == INVALID  # Y over X
     assert f(A, 64, A, A, A, A, A, A + 8192, 16, 4, 4, 1, 16, 64, 4, None) == INVALID  # unknown flag
+
+
+def test_w4a4_sizes_and_validation():
+    L = nv.lib
+    assert L.nvfp4_w4a4_weight_scales_bytes(300, 512) == 384 * 32
+    assert L.nvfp4_w4a4_x_scales_bytes(300, 512) == 512 * 32
+    assert L.nvfp4_w4a4_x_scales_bytes(300, 500) == 0
+    assert L.nvfp4_w4a4_workspace_size(300, 512) == 300 * 256 + 512 * 32 + 16
+    assert L.nvfp4_w4a4_weight_scales_bytes(1, 256) == 128 * 16
+    # K must be a multiple of 256
+    assert L.nvfp4_w4a4_prepare_weights(A, 16, 128, A + 65536, None) == SHAPE
+    assert L.nvfp4_w4a4_quantize_x(A, 128, 4, 128, A + 8192, A + 16384, A + 32768, 0, None) == SHAPE
+    assert L.nvfp4_w4a4_gemm(A, A, A, A, A, A, A, 16, 4, 16, 128, 0, None) == SHAPE
+    # no-ops need no device
+    assert L.nvfp4_w4a4_prepare_weights(A, 0, 256, A + 65536, None) == OK
+    assert L.nvfp4_w4a4_quantize_x(A, 256, 0, 256, A, A, A, 0, None) == OK
+    assert L.nvfp4_w4a4_gemm(A, A, A, A, A, A, A, 16, 0, 16, 256, 0, None) == OK
+    # null, alignment, overlap, flags
+    assert L.nvfp4_w4a4_prepare_weights(None, 16, 256, A, None) == INVALID
+    assert L.nvfp4_w4a4_prepare_weights(A, 16, 256, A + 8, None) == ALIGN
+    assert L.nvfp4_w4a4_prepare_weights(A, 16, 256, A + 64, None) == INVALID          # s_mma overlaps s
+    assert L.nvfp4_w4a4_quantize_x(A, 256, 4, 256, A + 8192, A + 16384, A + 32768, 4, None) == INVALID
+    assert L.nvfp4_w4a4_quantize_x(A, 128, 4, 256, A + 8192, A + 16384, A + 32768, 0, None) == INVALID  # ldx < K
+    assert L.nvfp4_w4a4_quantize_x(A, 260, 4, 256, A + 8192, A + 16384, A + 32768, 0, None) == ALIGN
+    assert L.nvfp4_w4a4_quantize_x(A, 256, 4, 256, A + 16, A + 16384, A + 32768, 0, None) == INVALID   # qx in X
+    assert L.nvfp4_w4a4_quantize_x(A, 256, 4, 256, A + 8192, A + 16384, A + 32770, 0, None) == ALIGN
+    assert L.nvfp4_w4a4_gemm(A, A + 4096, A + 8192, A + 16384, A + 32768, A + 65536, A + 131072, 8, 4, 16, 256,
+                             0, None) == INVALID                                       # ldy < N
+    assert L.nvfp4_w4a4_gemm(A, A + 4096, A + 8192, A + 16384, A + 32768, A + 65536, A + 16, 16, 4, 16, 256,
+                             0, None) == INVALID                                       # Y over qx
+    assert L.nvfp4_w4a4_gemm(A, A + 4096, A + 8192, A + 16384, A + 32768, A + 65536, A + 131072, 16, 4, 16, 256,
+                             8, None) == INVALID                                       # unknown flag
+    assert L.nvfp4_w4a4_linear(A, 256, None, A + 16384, A + 32768, A + 65536, A + 131072, 16, 4, 16, 256,
+                               None, 0, 0, None) == 6                                  # workspace missing
+    assert L.nvfp4_w4a4_linear(A, 256, None, A + 16384, A + 32768, A + 65536, A + 131072, 16, 4, 16, 256,
+                               A + 8, 1 << 20, 0, None) == ALIGN
