@@ -61,6 +61,14 @@ def mx_quantize_bytes(N: int, K: int) -> int:
     return 2 * N * K + N * K // 2 + N * K // 32
 
 
+def w4a4_gemm_bytes(M: int, N: int, K: int) -> int:
+    """W4A4 GEMM kernel alone: weight nibbles + scales, activation nibbles +
+    scales, Y, g and x_amax."""
+    return N * K // 2 + N * K // 16 + M * K // 2 + M * K // 16 + 2 * M * N + 8
+
+
+FP4_PER_BF16 = 4  # nominal dense FP4 / BF16 tensor throughput of B200 (9 / 2.25 PFLOP/s)
+
 MOE = {"E": 128, "N": 1536, "K": 2048, "top": 8}  # synthetic MoE layer: stacked experts, top-8 routing, one token
 
 
@@ -100,6 +108,9 @@ KERNEL_SOURCES = {
     "mx_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
     "moe_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "w4a4_m512": [_CSRC + "gemm_w4a4.cu", _CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh",
+                  _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "w4a4_gemm": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
 }
 
 
@@ -299,6 +310,24 @@ def run_gpu(args):
         nv.amax(wq_in, amax_buf)
         nv.quantize(wq_in, qq, sq, gq, amax=amax_buf)
 
+    # W4A4 prefill (NVFP4 activations): the same 8 weight copies, scales
+    # rearranged once for the block-scaled tensor cores
+    w4_ok = args.only in ("all", "w4a4_m512", "w4a4_gemm")
+    if w4_ok:
+        smmas = [nv.w4a4_prepare_weights(ss[i], K) for i in range(copies)]
+        ws_w4 = torch.empty((nv.w4a4_workspace_size(512, K),), dtype=torch.uint8, device=dev)
+        w4_amax = torch.empty((1,), dtype=torch.float32, device=dev)
+        w4_qx, w4_sx = nv.w4a4_quantize_x(X512, w4_amax)
+        Y512w = torch.empty((512, N), dtype=torch.bfloat16, device=dev)
+
+        def w4a4_all():  # activation amax + quantize + GEMM per call
+            for i in range(copies):
+                nv.w4a4_linear(X512, qs[i], smmas[i], g0, Y512w, ws_w4, static_weights=True)
+
+        def w4a4_gemm_all():  # the GEMM kernel alone on quantized activations
+            for i in range(copies):
+                nv.w4a4_gemm(w4_qx, w4_sx, w4_amax, qs[i], smmas[i], g0, Y512w, static_weights=True)
+
     rows.append(("quantize", quant_all, 1, 2))
     rows.append(("mx_quantize", mx_quant_all, 1, 1))
     if gemm_ok:
@@ -311,6 +340,10 @@ def run_gpu(args):
                 nv.gemm(X512, qs[i], ss[i], g0, Y512, workspace=ws512, static_weights=True)
 
         rows.append(("gemm_m512", m512_all, copies, 2))
+    if w4_ok:
+        rows.append(("w4a4_m512", w4a4_all, copies, 3))  # amax + quantize X + GEMM per call
+        rows.append(("w4a4_gemm", w4a4_gemm_all, copies, 1))
+    if gemm_ok:
         rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
     rows.append(("mx_gemv", mx_gemv_all, copies, 1))
     rows.append(("moe_gemv", moe_all, copies, 1))
@@ -432,6 +465,19 @@ def run_gpu(args):
         elif not gemm_ok and args.only == "all":
             kernels[name] = {"unavailable": gemm_err}
 
+    fp4_peak = bf16_burst * FP4_PER_BF16
+    for name in ("w4a4_m512", "w4a4_gemm"):
+        if name in per_launch_ms:
+            t = per_launch_ms[name] * 1e-3
+            fl = 2.0 * 512 * N * K
+            byt = gemm_bytes(512, N, K) if name == "w4a4_m512" else w4a4_gemm_bytes(512, N, K)
+            kernels[name] = {"us": t * 1e6, "TFLOP/s": fl / t / 1e12, "frac_fp4": fl / t / 1e12 / fp4_peak,
+                             "fp4_peak_tflops": fp4_peak,
+                             "fp4_peak_source": f"{peaks['source']} bf16 x {FP4_PER_BF16} (nominal dense FP4/BF16)",
+                             "GB/s": byt / t / 1e9, "frac_hbm": byt / t / 1e9 / hbm, "bytes": byt,
+                             "what": ("activation amax + NVFP4 quantize of X + block-scaled FP4 GEMM"
+                                      if name == "w4a4_m512" else "block-scaled FP4 GEMM on quantized X")}
+
     # ---- end to end through the public API with host buffers (decode GEMV):
     # pinned x -> device, GEMV, y -> pinned host, every step.
     x_host = workloads.activations(1, K, 1).reshape(-1).pin_memory()
@@ -479,9 +525,9 @@ def run_gpu(args):
             "config": {"workload": WORKLOAD, "N": N, "K": K, "M": 1, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {copies} rotating weight copies "
                              f"({copies * (N * K // 2 + N * K // 16) / 1e6:.0f} MB) per graph",
-                       "row_order": "quantize, MXFP4 quantize (each followed by an untimed read of 2 x L2 that writes back their dirty output), gemm M=512, gemm M=32, MXFP4 gemv, MoE gemv, gemv ordered, gemv static: each GEMV graph "
+                       "row_order": "quantize, MXFP4 quantize (each followed by an untimed read of 2 x L2 that writes back their dirty output), gemm M=512, W4A4 M=512 (step), W4A4 GEMM, gemm M=32, MXFP4 gemv, MoE gemv, gemv ordered, gemv static: each GEMV graph "
                                     "follows GEMVs, not the rows that leave tens of MB of dirty output in L2",
-                       "step": "quantize [17408,5120] (NVFP4, MXFP4) + gemm M=512 + gemm M=32 + MXFP4 gemv + grouped MoE gemv + gemv M=1 (x2: ordered and static-weights)",
+                       "step": "quantize [17408,5120] (NVFP4, MXFP4) + gemm M=512 + W4A4 M=512 (quantize X + GEMM) + W4A4 GEMM + gemm M=32 + MXFP4 gemv + grouped MoE gemv + gemv M=1 (x2: ordered and static-weights)",
             "gemv_launch": "8 GEMVs per graph on 8 weight copies, programmatic dependent launch (static weights)"},
             "roofline": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemv_gbs / hbm, "traffic": traffic,
@@ -576,7 +622,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=17408)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "gemm_m32",
-                                                      "gemm_m512", "mx_gemv", "mx_quantize", "moe_gemv"],
+                                                      "gemm_m512", "mx_gemv", "mx_quantize", "moe_gemv",
+                                                      "w4a4_m512", "w4a4_gemm"],
                     help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
