@@ -316,7 +316,7 @@ def run_gpu(args):
     if w4_ok:
         smmas = [nv.w4a4_prepare_weights(ss[i], K) for i in range(copies)]
         ws_w4 = torch.empty((nv.w4a4_workspace_size(512, K),), dtype=torch.uint8, device=dev)
-        w4_amax = torch.empty((1,), dtype=torch.float32, device=dev)
+        w4_amax = torch.empty((nv.AMAX_FLOATS,), dtype=torch.float32, device=dev)
         w4_qx, w4_sx = nv.w4a4_quantize_x(X512, w4_amax)
         Y512w = torch.empty((512, N), dtype=torch.bfloat16, device=dev)
 

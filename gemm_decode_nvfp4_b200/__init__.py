@@ -24,7 +24,7 @@ __all__ = [
     "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
     "mx_quantize", "mx_quantize_new", "mx_gemv", "gemv_grouped", "mx_to_nvfp4",
     "GIVEN_AMAX", "w4a4_prepare_weights", "w4a4_quantize_x", "w4a4_gemm", "w4a4_linear",
-    "w4a4_workspace_size",
+    "w4a4_workspace_size", "AMAX_FLOATS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -349,6 +349,7 @@ def mx_to_nvfp4(q: torch.Tensor, s_mx: torch.Tensor, stream=None):
 # weights' rule, block-scaled FP4 tensor-core GEMM.
 
 GIVEN_AMAX = 2  # NVFP4_W4A4_GIVEN_AMAX
+AMAX_FLOATS = 260  # NVFP4_W4A4_AMAX_FLOATS: the x_amax buffer of a dynamic quantize
 
 
 def w4a4_prepare_weights(s: torch.Tensor, K: int, stream=None) -> torch.Tensor:
@@ -363,10 +364,13 @@ def w4a4_prepare_weights(s: torch.Tensor, K: int, stream=None) -> torch.Tensor:
 
 
 def w4a4_quantize_x(X: torch.Tensor, x_amax: torch.Tensor, given_amax: bool = False, stream=None):
-    """X [M, K] -> (qx [M, K/2], sx in the tensor-core scale layout); x_amax [1]
-    receives max |X| unless given_amax."""
+    """X [M, K] -> (qx [M, K/2], sx in the tensor-core scale layout).  x_amax:
+    given_amax: [1] (or longer), read; else [AMAX_FLOATS], x_amax[0] receives
+    max |X|."""
     _need(X, torch.bfloat16, "X", 2)
     _need(x_amax, torch.float32, "x_amax")
+    if not given_amax and x_amax.numel() < AMAX_FLOATS:
+        raise ValueError(f"x_amax needs {AMAX_FLOATS} floats for a dynamic amax")
     M, K = X.shape
     if X.stride(1) != 1:
         raise ValueError("X rows must be contiguous")

@@ -393,7 +393,7 @@ size_t nvfp4_w4a4_x_scales_bytes(int64_t M, int64_t K) {
 
 size_t nvfp4_w4a4_workspace_size(int64_t M, int64_t K) {
   if (M <= 0 || K <= 0 || K % 256) return 0;
-  return round_up((size_t)(M * K / 2), 16) + nvfp4_w4a4_x_scales_bytes(M, K) + 16;
+  return round_up((size_t)(M * K / 2), 16) + nvfp4_w4a4_x_scales_bytes(M, K) + NVFP4_W4A4_AMAX_FLOATS * 4;
 }
 
 nvfp4_status nvfp4_w4a4_prepare_weights(const uint8_t* s, int64_t N, int64_t K, uint8_t* s_mma,
@@ -422,21 +422,16 @@ nvfp4_status nvfp4_w4a4_quantize_x(const uint16_t* X, int64_t ldx, int64_t M, in
   if (ldx < K) return fail(NVFP4_ERR_INVALID_ARG, "ldx=%lld < K=%lld", (long long)ldx, (long long)K);
   if (!aligned16(X) || !aligned16(qx) || !aligned16(sx) || ldx % 8 || !aligned4(x_amax))
     return fail(NVFP4_ERR_ALIGNMENT, "X, qx, sx must be 16-byte aligned, ldx a multiple of 8, x_amax 4-byte aligned");
+  const bool given = (flags & NVFP4_W4A4_GIVEN_AMAX) != 0;
   const size_t xb = (size_t)((M - 1) * ldx + K) * 2, qb = (size_t)(M * K / 2), sb = nvfp4_w4a4_x_scales_bytes(M, K);
-  if (overlaps(X, xb, qx, qb) || overlaps(X, xb, sx, sb) || overlaps(qx, qb, sx, sb) || overlaps(x_amax, 4, X, xb) ||
-      overlaps(x_amax, 4, qx, qb) || overlaps(x_amax, 4, sx, sb))
+  const size_t ab = given ? 4 : NVFP4_W4A4_AMAX_FLOATS * 4;
+  if (overlaps(X, xb, qx, qb) || overlaps(X, xb, sx, sb) || overlaps(qx, qb, sx, sb) || overlaps(x_amax, ab, X, xb) ||
+      overlaps(x_amax, ab, qx, qb) || overlaps(x_amax, ab, sx, sb))
     return fail(NVFP4_ERR_INVALID_ARG, "X, qx, sx and x_amax must not overlap");
   int sms = 0;
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
-  cudaStream_t cs = (cudaStream_t)stream;
-  cudaError_t e = cudaSuccess;
-  if (!(flags & NVFP4_W4A4_GIVEN_AMAX)) {
-    e = cudaMemsetAsync(x_amax, 0, sizeof(float), cs);
-    if (e == cudaSuccess) e = nvfp4::launch_amax(X, M, K, ldx, x_amax, cs, sms);
-    if (e != cudaSuccess) return cuda_fail(e, "activation amax launch");
-  }
-  e = nvfp4::launch_quantize_x_mma(X, ldx, M, K, x_amax, qx, sx, cs, sms);
+  cudaError_t e = nvfp4::launch_quantize_x_mma(X, ldx, M, K, x_amax, given, qx, sx, (cudaStream_t)stream, sms);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "activation quantize launch");
 }
 
@@ -488,7 +483,7 @@ nvfp4_status nvfp4_w4a4_linear(const uint16_t* X, int64_t ldx, const float* x_am
   }
   uint8_t* qx = static_cast<uint8_t*>(workspace);
   uint8_t* sx = qx + round_up((size_t)(M * K / 2), 16);
-  // the dynamic amax goes to the workspace's last slot; a given one is only read
+  // the dynamic amax (and its per-CTA maxima) goes to the workspace's end; a given one is only read
   float* amax = x_amax ? const_cast<float*>(x_amax) : reinterpret_cast<float*>(sx + nvfp4_w4a4_x_scales_bytes(M, K));
   st = nvfp4_w4a4_quantize_x(X, ldx, M, K, qx, sx, amax, x_amax ? NVFP4_W4A4_GIVEN_AMAX : 0u, stream);
   if (st != NVFP4_OK) return st;

@@ -41,7 +41,9 @@ cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count);
 // rows padded with zero scales to a multiple of 256); the weight scales
 // rearranged once into the same layout (rows padded to a multiple of 128);
 // the block-scaled FP4 GEMM Y = bf16(g * g_x * sum sx sw qx qw).
-cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, const float* x_amax,
+// amax: given ? amax[0] is read : amax[0] receives max |X| and amax[1 .. 256]
+// hold per-CTA partial maxima (NVFP4_W4A4_AMAX_FLOATS floats in all).
+cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, float* amax, bool given,
                                   uint8_t* qx, uint8_t* sx, cudaStream_t stream, int sms);
 cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t* s_mma, cudaStream_t stream,
                                  int sms);

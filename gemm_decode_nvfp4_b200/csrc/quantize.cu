@@ -97,6 +97,18 @@ __device__ __forceinline__ void quantize_block(const float (&f)[16], float g, ui
   codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
 }
 
+// Quantize the 16 BF16 values of (v0, v1): scale byte and 8 code bytes.
+__device__ __forceinline__ void quantize_store_regs(uint4 v0, uint4 v1, float g, uint32_t& sc, uint2& codes) {
+  const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  float f[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = bf16lo_to_float(wv[i]);
+    f[2 * i + 1] = bf16hi_to_float(wv[i]);
+  }
+  quantize_block(f, g, sc, codes);
+}
+
 // Quantize the 16 BF16 values of (v0, v1) and store 8 code bytes and the scale.
 __device__ __forceinline__ void quantize_store(uint4 v0, uint4 v1, float g, uint8_t* qd, uint8_t* sd) {
   const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -243,50 +255,75 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
 //
 // X [M, K] quantized by the weights' rule with g_x = x_amax / 2688: codes
 // row-major [M, K/2] and the E4M3 scales in the tensor core's scale-factor
-// layout: for row m and 64-element step kk, the four scale bytes of its
-// 16-blocks form one 32-bit word at byte
-//   ((m / 128) * (K / 64) + kk) * 512 + (m % 32) * 16 + ((m % 128) / 32) * 4,
+// layout: the scale of row m, 16-block b sits at byte
+//   ((m / 128) * (K / 64) + b / 4) * 512 + (m % 32) * 16 + ((m % 128) / 32) * 4 + b % 4,
 // i.e. one 512-byte atom per 128 rows and 64 k.  Rows M .. Mpad-1 get zero
 // scales (Mpad = M rounded up to 256, the GEMM's token tile).
-__global__ void __launch_bounds__(256) quantize_x_mma_kernel(const uint16_t* __restrict__ X, int64_t ldx,
-                                                             int64_t M, int64_t K, int64_t Mpad,
-                                                             const float* __restrict__ x_amax,
-                                                             uint8_t* __restrict__ qx, uint8_t* __restrict__ sx) {
+//
+// The dynamic amax takes two launches and no memset: x_amax_partial_kernel
+// writes one maximum per CTA into amax[1 ..], and every CTA of the quantizer
+// reduces those before it starts (CTA 0 also stores the total in amax[0]).
+constexpr int kXAmaxParts = 256;
+
+__global__ void __launch_bounds__(256) x_amax_partial_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t M,
+                                                             int64_t K, float* __restrict__ amax) {
+  __shared__ float red[8];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const float g = __fdiv_rn(*x_amax, 2688.0f);
-  const int64_t steps = K / 64;
-  const int64_t total = Mpad * steps;
+  const int64_t vpr = K / 8, total = M * vpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  float m = 0.0f;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
+    const int64_t r = t / vpr, c = (t - r * vpr) * 8;
+    m = absmax8(ld_stream_v4(X + r * ldx + c), m);
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+    amax[1 + blockIdx.x] = m;
+  }
+}
+
+// One thread per (row, 16-block) of the padded rows.  parts > 0: reduce
+// amax[1 .. parts] first (dynamic); parts == 0: amax[0] is given.
+__global__ void __launch_bounds__(256) quantize_x_mma_kernel(const uint16_t* __restrict__ X, int64_t ldx,
+                                                             int64_t M, int64_t K, int64_t Mpad,
+                                                             float* __restrict__ amax, int parts,
+                                                             uint8_t* __restrict__ qx, uint8_t* __restrict__ sx) {
+  __shared__ float s_amax;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x < 32) {
+    float m = 0.0f;
+    if (parts > 0) {
+      for (int i = threadIdx.x; i < parts; i += 32) m = fmaxf(m, amax[1 + i]);
+      m = warp_max(m);
+    } else {
+      m = amax[0];
+    }
+    if (threadIdx.x == 0) {
+      s_amax = m;
+      if (parts > 0 && blockIdx.x == 0) amax[0] = m;
+    }
+  }
+  __syncthreads();
+  const float g = __fdiv_rn(s_amax, 2688.0f);
+  const int64_t nb = K / 16, steps = K / 64;
+  const int64_t total = Mpad * nb;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
-    const int64_t m = t / steps, kk = t - m * steps;
-    uint32_t word = 0;
+    const int64_t m = t / nb, b = t - m * nb;
+    uint32_t sc = 0;
     if (m < M) {
-      const uint4* src = reinterpret_cast<const uint4*>(X + m * ldx + kk * 64);
-      uint4 v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = ld_stream_v4(src + i);
-      uint2 codes[4];
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t wv[8] = {v[2 * b].x, v[2 * b].y, v[2 * b].z, v[2 * b].w,
-                                v[2 * b + 1].x, v[2 * b + 1].y, v[2 * b + 1].z, v[2 * b + 1].w};
-        float f[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          f[2 * i] = bf16lo_to_float(wv[i]);
-          f[2 * i + 1] = bf16hi_to_float(wv[i]);
-        }
-        uint32_t sc;
-        quantize_block(f, g, sc, codes[b]);
-        word |= sc << (8 * b);
-      }
-      uint4* dst = reinterpret_cast<uint4*>(qx + m * (K / 2) + kk * 32);
-      dst[0] = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
-      dst[1] = make_uint4(codes[2].x, codes[2].y, codes[3].x, codes[3].y);
+      const uint16_t* src = X + m * ldx + b * 16;
+      uint2 codes;
+      quantize_store_regs(ld_stream_v4(src), ld_stream_v4(src + 8), g, sc, codes);
+      *reinterpret_cast<uint2*>(qx + m * (K / 2) + b * 8) = codes;
     }
     const int64_t r = m % 128;
-    *reinterpret_cast<uint32_t*>(sx + ((m / 128) * steps + kk) * 512 + (r % 32) * 16 + (r / 32) * 4) = word;
+    sx[((m / 128) * steps + b / 4) * 512 + (r % 32) * 16 + (r / 32) * 4 + (b % 4)] = (uint8_t)sc;
   }
 }
 
@@ -382,22 +419,32 @@ cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, const float* x_amax,
+cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, float* amax, bool given,
                                   uint8_t* qx, uint8_t* sx, cudaStream_t stream, int sms) {
-  const int64_t Mpad = (M + 255) / 256 * 256;
-  const int grid = grid_for(Mpad * (K / 64), sms);
-  const int64_t ldx_ = ldx, M_ = M, K_ = K;
-  void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&Mpad, (void*)&x_amax, (void*)&qx,
-                  (void*)&sx};
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(256);
-  cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  int64_t ldx_ = ldx, M_ = M, K_ = K;
+  int parts = 0;
+  if (!given) {
+    const int64_t blocks = (M * (K / 8) + 255) / 256;
+    parts = (int)(blocks < kXAmaxParts ? blocks : kXAmaxParts);
+    cfg.gridDim = dim3(parts);
+    void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&amax};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, (const void*)x_amax_partial_kernel, args);
+    if (e != cudaSuccess) return e;
+  }
+  int64_t Mpad = (M + 255) / 256 * 256;
+  const int64_t blocks = (Mpad * (K / 16) + 255) / 256;
+  const int64_t cap = (int64_t)sms * 16;
+  cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
+  void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&Mpad, (void*)&amax, (void*)&parts,
+                  (void*)&qx, (void*)&sx};
   return cudaLaunchKernelExC(&cfg, (const void*)quantize_x_mma_kernel, args);
 }
 

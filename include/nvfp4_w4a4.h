@@ -44,6 +44,10 @@ extern "C" {
 /* x_amax is an input (a calibrated amax) instead of being computed from X. */
 #define NVFP4_W4A4_GIVEN_AMAX 2u
 
+/* Floats of the x_amax buffer of a dynamic-amax nvfp4_w4a4_quantize_x:
+ * element 0 receives max |X|, the rest holds per-CTA partial maxima. */
+#define NVFP4_W4A4_AMAX_FLOATS 260
+
 /* Bytes of the weight scales [N, K/16] in the MMA layout (rows padded to 128). */
 NVFP4_API size_t nvfp4_w4a4_weight_scales_bytes(int64_t N, int64_t K);
 
@@ -61,9 +65,10 @@ NVFP4_API nvfp4_status nvfp4_w4a4_prepare_weights(const uint8_t* s, int64_t N, i
 /*
  * Quantize X [M, K] for the W4A4 GEMM: codes qx [M, K/2] and scales sx in the
  * MMA layout (nvfp4_w4a4_x_scales_bytes(M, K) bytes).  Without
- * NVFP4_W4A4_GIVEN_AMAX in flags, *x_amax receives max |X| (it is zeroed and
- * reduced on the stream first); with it, *x_amax is read.  qx, sx and x_amax
- * must not overlap X or each other.  M == 0 is a no-op.
+ * NVFP4_W4A4_GIVEN_AMAX in flags, x_amax points to NVFP4_W4A4_AMAX_FLOATS
+ * floats and x_amax[0] receives max |X| (two kernels: per-CTA maxima, then the
+ * quantizer, which reduces them); with it, only x_amax[0] is read.  qx, sx and
+ * the x_amax floats must not overlap X or each other.  M == 0 is a no-op.
  */
 NVFP4_API nvfp4_status nvfp4_w4a4_quantize_x(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, uint8_t* qx,
                                              uint8_t* sx, float* x_amax, uint32_t flags, nvfp4_stream_t stream);
@@ -78,7 +83,7 @@ NVFP4_API nvfp4_status nvfp4_w4a4_gemm(const uint8_t* qx, const uint8_t* sx, con
                                        const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M,
                                        int64_t N, int64_t K, uint32_t flags, nvfp4_stream_t stream);
 
-/* Workspace of nvfp4_w4a4_linear: qx, sx and the x_amax slot, 16-byte aligned. */
+/* Workspace of nvfp4_w4a4_linear: qx, sx and the dynamic x_amax floats. */
 NVFP4_API size_t nvfp4_w4a4_workspace_size(int64_t M, int64_t K);
 
 /*

@@ -119,7 +119,7 @@ def test_w4a4_sizes_and_validation():
     assert L.nvfp4_w4a4_weight_scales_bytes(300, 512) == 384 * 32
     assert L.nvfp4_w4a4_x_scales_bytes(300, 512) == 512 * 32
     assert L.nvfp4_w4a4_x_scales_bytes(300, 500) == 0
-    assert L.nvfp4_w4a4_workspace_size(300, 512) == 300 * 256 + 512 * 32 + 16
+    assert L.nvfp4_w4a4_workspace_size(300, 512) == 300 * 256 + 512 * 32 + 260 * 4
     assert L.nvfp4_w4a4_weight_scales_bytes(1, 256) == 128 * 16
     # K must be a multiple of 256
     assert L.nvfp4_w4a4_prepare_weights(A, 16, 128, A + 65536, None) == SHAPE
@@ -148,3 +148,11 @@ def test_w4a4_sizes_and_validation():
                                None, 0, 0, None) == 6                                  # workspace missing
     assert L.nvfp4_w4a4_linear(A, 256, None, A + 16384, A + 32768, A + 65536, A + 131072, 16, 4, 16, 256,
                                A + 8, 1 << 20, 0, None) == ALIGN
+
+
+def test_w4a4_binding_constants_match_header():
+    import re
+    with open(nv.W4A4_HEADER_PATH) as f:
+        text = f.read()
+    assert int(re.search(r"#define NVFP4_W4A4_AMAX_FLOATS (\d+)", text).group(1)) == nv.AMAX_FLOATS
+    assert int(re.search(r"#define NVFP4_W4A4_GIVEN_AMAX (\d+)u", text).group(1)) == nv.GIVEN_AMAX

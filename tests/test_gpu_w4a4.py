@@ -63,11 +63,11 @@ def test_prepare_weights_layout(nv, N, K):
 @pytest.mark.parametrize("M,K", [(512, 5120), (300, 512), (1, 256), (257, 1024)])
 def test_quantize_x_bit_exact(nv, M, K):
     X = workloads.activations(M, K, M + K)
-    amax = torch.empty((1,), dtype=torch.float32, device="cuda")
+    amax = torch.empty((nv.AMAX_FLOATS,), dtype=torch.float32, device="cuda")
     qx, sx = nv.w4a4_quantize_x(X.cuda(), amax)
     torch.cuda.synchronize()
     q_ref, s_ref, g_ref = oracle.quantize(X, oracle.tensor_scale(oracle.amax(X)))
-    assert amax.item() == float(oracle.amax(X))
+    assert amax[0].item() == float(oracle.amax(X))
     assert np.array_equal(qx.cpu().numpy(), q_ref)
     got = from_mma_layout(sx.cpu().numpy(), M, K, 256)
     assert np.array_equal(got[:M], s_ref) and not got[M:].any()
