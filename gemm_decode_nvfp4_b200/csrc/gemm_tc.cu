@@ -33,8 +33,6 @@
 //   - warp 1, one thread: tcgen05.mma into the TMEM accumulator [128, BNT],
 //     committing each stage to its "empty" barrier;
 //   - warps 2..9 then read TMEM, apply g * 2^-e_m and store BF16 Y.
-// Each CTA walks K from its own offset (weight tile index mod K/256), which
-// spreads the reads of the shared X' tile over L2.
 // Kernels are launched with programmatic dependent launch: with static
 // weights the W tiles start streaming while the previous kernel (the X prep)
 // is still running; X', e_m and Y are touched only after it completes.
@@ -354,29 +352,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // Weight stage wb holds the k range of chunk (wb + rot) % num_wb, and MMA
-      // stage kb the matching 64 k: CTAs of neighbouring weight tiles start at
-      // different k, so that the CTAs sharing the X' tile do not all read the
-      // same bytes of it at once.
-      const int rot = blockIdx.x % num_wb;
-      auto chunk = [&](int wb) { return wb + rot < num_wb ? wb + rot : wb + rot - num_wb; };
       auto issue_w = [&](int wb) {
-        const int ws = wb % NW, wc = chunk(wb);
+        const int ws = wb % NW;
         ptx::mbar_arrive_expect_tx(&bars->wfull[ws], C::kWBytes + C::kSBytes);
-        ptx::tma_load_2d(w_tile(ws), &tmap_w, &bars->wfull[ws], wc * 128, n0);
-        ptx::tma_load_2d(s_tile(ws), &tmap_s, &bars->wfull[ws], wc * 16, n0);
+        ptx::tma_load_2d(w_tile(ws), &tmap_w, &bars->wfull[ws], wb * 128, n0);
+        ptx::tma_load_2d(s_tile(ws), &tmap_s, &bars->wfull[ws], wb * 16, n0);
       };
       auto issue_x = [&](int xb) {
         const int xs = xb % NX;
         ptx::mbar_arrive_expect_tx(&bars->xfull[xs], C::kXBytes);
 #pragma unroll
-        for (int i = 0; i < XG; ++i) {
-          const int kb = xb * XG + i;
-          const int kx = (chunk(kb / 4) * 4 + kb % 4) * kBK;
+        for (int i = 0; i < XG; ++i)
 #pragma unroll
           for (int h = 0; h < (BNT + 255) / 256; ++h)
-            ptx::tma_load_2d(x_slot(xs) + i * C::kXSub + h * 256 * 128, &tmap_x, &bars->xfull[xs], kx, m0 + h * 256);
-        }
+            ptx::tma_load_2d(x_slot(xs) + i * C::kXSub + h * 256 * 128, &tmap_x, &bars->xfull[xs],
+                             (xb * XG + i) * kBK, m0 + h * 256);
       };
       // weight stages that need no slot release go out before the X prep ends
       const int w_first = num_wb < NW ? num_wb : NW;

@@ -29,9 +29,7 @@
 //   - warps 2..5: the epilogue, TMEM -> g * g_x -> BF16 Y through shared memory.
 // A stage's TMEM scale columns are rewritten only after the MMAs that read
 // them have completed (the stage's empty barrier), and tcgen05.cp is ordered
-// before the MMAs its thread issues after it.  Each CTA walks K starting at
-// its own offset (weight tile index mod K/256), which spreads the reads of the
-// shared token tile over L2.  Every wait is bounded.
+// before the MMAs its thread issues after it.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -168,21 +166,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* sa_src = s_mma + (int64_t)nt * steps64 * 512;
       const uint8_t* sb_src0 = sx + (int64_t)(2 * mt) * steps64 * 512;
       const uint8_t* sb_src1 = sx + (int64_t)(2 * mt + 1) * steps64 * 512;
-      // Stage ks holds the k range of chunk (ks + rot) % num_ks: CTAs of
-      // neighbouring weight tiles start at different k, so that the 100+ CTAs
-      // sharing a token tile do not all read the same bytes of it at once.
-      const int rot = nt % num_ks;
-      auto chunk = [&](int ks) { return ks + rot < num_ks ? ks + rot : ks + rot - num_ks; };
       auto issue_w = [&](int ks) {
-        const int st = ks % kStages, kc = chunk(ks);
-        ptx::tma_load_2d(a_tile(st), &tmap_w, &bars->full[st], kc * 128, n0);
-        ptx::bulk_load(sfa(st), sa_src + kc * kSFABytes, kSFABytes, &bars->full[st]);
+        const int st = ks % kStages;
+        ptx::tma_load_2d(a_tile(st), &tmap_w, &bars->full[st], ks * 128, n0);
+        ptx::bulk_load(sfa(st), sa_src + ks * kSFABytes, kSFABytes, &bars->full[st]);
       };
       auto issue_x = [&](int ks) {
-        const int st = ks % kStages, kc = chunk(ks);
-        ptx::tma_load_2d(b_tile(st), &tmap_x, &bars->full[st], kc * 128, m0);
-        ptx::bulk_load(sfb(st), sb_src0 + kc * 2048, 2048, &bars->full[st]);
-        ptx::bulk_load(sfb(st) + 2048, sb_src1 + kc * 2048, 2048, &bars->full[st]);
+        const int st = ks % kStages;
+        ptx::tma_load_2d(b_tile(st), &tmap_x, &bars->full[st], ks * 128, m0);
+        ptx::bulk_load(sfb(st), sb_src0 + ks * 2048, 2048, &bars->full[st]);
+        ptx::bulk_load(sfb(st) + 2048, sb_src1 + ks * 2048, 2048, &bars->full[st]);
       };
       // static weights: the first stages' weights stream before the producer
       // of X has finished
