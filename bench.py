@@ -101,16 +101,17 @@ def kernel_source_hash(files) -> str:
 _CSRC = "gemm_decode_nvfp4_b200/csrc/"
 KERNEL_SOURCES = {
     "gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
-    "quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
+    "quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh"],
     "gemm_m32": [_CSRC + "gemm_small.cu", _CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh",
                  _CSRC + "tc_host.h"],
     "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
     "mx_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
-    "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
+    "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh"],
     "moe_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
-    "w4a4_m512": [_CSRC + "gemm_w4a4.cu", _CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh",
+    "w4a4_m512": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
                   _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
-    "w4a4_gemm": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "w4a4_gemm": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
+                  _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
 }
 
 

@@ -8,7 +8,8 @@
 // Here:
 //   Y[m, n] = bf16(g * g_x * sum_k (sw[n, k/16] qw[n, k]) (sx[m, k/16] qx[m, k]))
 // with g_x = x_amax / 2688 and X quantized by the weights' rule
-// (quantize_x_mma_kernel).  Every product of two E2M1 codes and two E4M3
+// (x_amax_partial_kernel and quantize_x_mma_kernel below, with the block
+// rule of nvfp4_quant.cuh).  Every product of two E2M1 codes and two E4M3
 // scales is exact in fp32; the tensor core accumulates in fp32.
 //
 // Scale-factor layout (weights and activations alike): one 512-byte atom per
@@ -36,6 +37,7 @@
 
 #include "nvfp4_device.cuh"
 #include "nvfp4_kernels.h"
+#include "nvfp4_quant.cuh"
 #include "sm100_ptx.cuh"
 #include "tc_host.h"
 
@@ -279,6 +281,91 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------- activations for W4A4 GEMMs
+//
+// X [M, K] quantized by the weights' rule with g_x = x_amax / 2688: codes
+// row-major [M, K/2] and the E4M3 scales in the tensor core's scale-factor
+// layout: the scale of row m, 16-block b sits at byte
+//   ((m / 128) * (K / 64) + b / 4) * 512 + (m % 32) * 16 + ((m % 128) / 32) * 4 + b % 4,
+// i.e. one 512-byte atom per 128 rows and 64 k.  Rows M .. Mpad-1 get zero
+// scales (Mpad = M rounded up to 256, the GEMM's token tile).
+//
+// The dynamic amax takes two launches and no memset: x_amax_partial_kernel
+// writes one maximum per CTA into amax[1 ..], and every CTA of the quantizer
+// reduces those before it starts (CTA 0 also stores the total in amax[0]).
+constexpr int kXAmaxParts = 256;
+
+__global__ void __launch_bounds__(256) x_amax_partial_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t M,
+                                                             int64_t K, float* __restrict__ amax) {
+  __shared__ float red[8];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t vpr = K / 8, total = M * vpr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  float m = 0.0f;
+  // eight 16-byte loads in flight per thread (one memory round trip for
+  // tensors up to 8 x the grid's threads)
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += 8 * stride) {
+    uint4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t u = t + i * stride;
+      const int64_t r = u / vpr, c = (u - r * vpr) * 8;
+      v[i] = u < total ? ld_stream_v4(X + r * ldx + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = absmax8(v[i], m);
+  }
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
+    amax[1 + blockIdx.x] = m;
+  }
+}
+
+// One thread per (row, 16-block) of the padded rows.  parts > 0: reduce
+// amax[1 .. parts] first (dynamic); parts == 0: amax[0] is given.
+__global__ void __launch_bounds__(256) quantize_x_mma_kernel(const uint16_t* __restrict__ X, int64_t ldx,
+                                                             int64_t M, int64_t K, int64_t Mpad,
+                                                             float* __restrict__ amax, int parts,
+                                                             uint8_t* __restrict__ qx, uint8_t* __restrict__ sx) {
+  __shared__ float s_amax;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x < 32) {
+    float m = 0.0f;
+    if (parts > 0) {
+      for (int i = threadIdx.x; i < parts; i += 32) m = fmaxf(m, amax[1 + i]);
+      m = warp_max(m);
+    } else {
+      m = amax[0];
+    }
+    if (threadIdx.x == 0) {
+      s_amax = m;
+      if (parts > 0 && blockIdx.x == 0) amax[0] = m;
+    }
+  }
+  __syncthreads();
+  const float g = __fdiv_rn(s_amax, 2688.0f);
+  const int64_t nb = K / 16, steps = K / 64;
+  const int64_t total = Mpad * nb;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
+    const int64_t m = t / nb, b = t - m * nb;
+    uint32_t sc = 0;
+    if (m < M) {
+      const uint16_t* src = X + m * ldx + b * 16;
+      uint2 codes;
+      quantize_store_regs(ld_stream_v4(src), ld_stream_v4(src + 8), g, sc, codes);
+      *reinterpret_cast<uint2*>(qx + m * (K / 2) + b * 8) = codes;
+    }
+    const int64_t r = m % 128;
+    sx[((m / 128) * steps + b / 4) * 512 + (r % 32) * 16 + (r / 32) * 4 + (b % 4)] = (uint8_t)sc;
+  }
+}
+
 int grid_for(int64_t work_items, int sms) {
   const int64_t blocks = (work_items + 255) / 256;
   const int64_t cap = (int64_t)sms * 8;
@@ -286,6 +373,35 @@ int grid_for(int64_t work_items, int sms) {
 }
 
 }  // namespace
+
+cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, float* amax, bool given,
+                                  uint8_t* qx, uint8_t* sx, cudaStream_t stream, int sms) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int64_t ldx_ = ldx, M_ = M, K_ = K;
+  int parts = 0;
+  if (!given) {
+    const int64_t blocks = (M * (K / 8) + 255) / 256;
+    parts = (int)(blocks < kXAmaxParts ? blocks : kXAmaxParts);
+    cfg.gridDim = dim3(parts);
+    void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&amax};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, (const void*)x_amax_partial_kernel, args);
+    if (e != cudaSuccess) return e;
+  }
+  int64_t Mpad = (M + 255) / 256 * 256;
+  const int64_t blocks = (Mpad * (K / 16) + 255) / 256;
+  const int64_t cap = (int64_t)sms * 16;
+  cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
+  void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&Mpad, (void*)&amax, (void*)&parts,
+                  (void*)&qx, (void*)&sx};
+  return cudaLaunchKernelExC(&cfg, (const void*)quantize_x_mma_kernel, args);
+}
 
 cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t* s_mma, cudaStream_t stream,
                                  int sms) {

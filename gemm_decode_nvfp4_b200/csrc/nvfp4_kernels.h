@@ -35,7 +35,7 @@ cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q
                                 cudaStream_t stream);
 // Problems of grouped GEMVs whose ids were out of range since the last read.
 cudaError_t read_and_clear_gemv_bad_ids(unsigned int* count);
-// W4A4 (quantize.cu, gemm_w4a4.cu): X quantized by the weights' rule with
+// W4A4 (gemm_w4a4.cu): X quantized by the weights' rule with
 // g_x = *x_amax / 2688 into row-major codes qx [M, K/2] and scales sx in the
 // tensor core's scale-factor layout (512-byte atoms per 128 rows x 64 k,
 // rows padded with zero scales to a multiple of 256); the weight scales

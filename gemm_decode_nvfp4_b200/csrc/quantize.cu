@@ -12,26 +12,11 @@
 // that are contiguous across a warp and blocks never straddle threads.
 #include "nvfp4_kernels.h"
 #include "nvfp4_device.cuh"
+#include "nvfp4_quant.cuh"
 
 namespace nvfp4 {
 
 namespace {
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
-
-__device__ __forceinline__ float absmax8(uint4 v, float m) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = fmaxf(m, fabsf(bf16lo_to_float(w[i])));
-    m = fmaxf(m, fabsf(bf16hi_to_float(w[i])));
-  }
-  return m;
-}
 
 // amax over rows x cols (cols % 8 == 0), atomically max-merged into *out.
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ w, int64_t rows,
@@ -67,46 +52,6 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     // non-negative floats order like their bit patterns
     if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(m));
   }
-}
-
-// One 16-element block: scale byte and 8 code bytes.
-__device__ __forceinline__ void quantize_block(const float (&f)[16], float g, uint32_t& scale,
-                                               uint2& codes) {
-  float amax_b = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(f[i]));
-  uint32_t sc = 0;
-  if (g != 0.0f) sc = float_to_e4m3_satfinite(__fdiv_rn(__fdiv_rn(amax_b, 6.0f), g));
-  const float d = __fmul_rn(e4m3_to_float(sc), g);
-  uint32_t c[8];
-  if (d == 0.0f) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = 0;
-  } else {
-    const float r = __frcp_rn(d);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      // +-0 keeps its sign even when r overflowed to infinity
-      const float lo = (f[2 * i] == 0.0f) ? f[2 * i] : __fmul_rn(f[2 * i], r);
-      const float hi = (f[2 * i + 1] == 0.0f) ? f[2 * i + 1] : __fmul_rn(f[2 * i + 1], r);
-      c[i] = float2_to_e2m1x2_satfinite(lo, hi);
-    }
-  }
-  scale = sc;
-  codes.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-  codes.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-}
-
-// Quantize the 16 BF16 values of (v0, v1): scale byte and 8 code bytes.
-__device__ __forceinline__ void quantize_store_regs(uint4 v0, uint4 v1, float g, uint32_t& sc, uint2& codes) {
-  const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-  float f[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    f[2 * i] = bf16lo_to_float(wv[i]);
-    f[2 * i + 1] = bf16hi_to_float(wv[i]);
-  }
-  quantize_block(f, g, sc, codes);
 }
 
 // Quantize the 16 BF16 values of (v0, v1) and store 8 code bytes and the scale.
@@ -251,82 +196,6 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const uint16_t* __rest
   }
 }
 
-// ------------------------------------------------- activations for W4A4 GEMMs
-//
-// X [M, K] quantized by the weights' rule with g_x = x_amax / 2688: codes
-// row-major [M, K/2] and the E4M3 scales in the tensor core's scale-factor
-// layout: the scale of row m, 16-block b sits at byte
-//   ((m / 128) * (K / 64) + b / 4) * 512 + (m % 32) * 16 + ((m % 128) / 32) * 4 + b % 4,
-// i.e. one 512-byte atom per 128 rows and 64 k.  Rows M .. Mpad-1 get zero
-// scales (Mpad = M rounded up to 256, the GEMM's token tile).
-//
-// The dynamic amax takes two launches and no memset: x_amax_partial_kernel
-// writes one maximum per CTA into amax[1 ..], and every CTA of the quantizer
-// reduces those before it starts (CTA 0 also stores the total in amax[0]).
-constexpr int kXAmaxParts = 256;
-
-__global__ void __launch_bounds__(256) x_amax_partial_kernel(const uint16_t* __restrict__ X, int64_t ldx, int64_t M,
-                                                             int64_t K, float* __restrict__ amax) {
-  __shared__ float red[8];
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int64_t vpr = K / 8, total = M * vpr;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  float m = 0.0f;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
-    const int64_t r = t / vpr, c = (t - r * vpr) * 8;
-    m = absmax8(ld_stream_v4(X + r * ldx + c), m);
-  }
-  m = warp_max(m);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
-    amax[1 + blockIdx.x] = m;
-  }
-}
-
-// One thread per (row, 16-block) of the padded rows.  parts > 0: reduce
-// amax[1 .. parts] first (dynamic); parts == 0: amax[0] is given.
-__global__ void __launch_bounds__(256) quantize_x_mma_kernel(const uint16_t* __restrict__ X, int64_t ldx,
-                                                             int64_t M, int64_t K, int64_t Mpad,
-                                                             float* __restrict__ amax, int parts,
-                                                             uint8_t* __restrict__ qx, uint8_t* __restrict__ sx) {
-  __shared__ float s_amax;
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (threadIdx.x < 32) {
-    float m = 0.0f;
-    if (parts > 0) {
-      for (int i = threadIdx.x; i < parts; i += 32) m = fmaxf(m, amax[1 + i]);
-      m = warp_max(m);
-    } else {
-      m = amax[0];
-    }
-    if (threadIdx.x == 0) {
-      s_amax = m;
-      if (parts > 0 && blockIdx.x == 0) amax[0] = m;
-    }
-  }
-  __syncthreads();
-  const float g = __fdiv_rn(s_amax, 2688.0f);
-  const int64_t nb = K / 16, steps = K / 64;
-  const int64_t total = Mpad * nb;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += stride) {
-    const int64_t m = t / nb, b = t - m * nb;
-    uint32_t sc = 0;
-    if (m < M) {
-      const uint16_t* src = X + m * ldx + b * 16;
-      uint2 codes;
-      quantize_store_regs(ld_stream_v4(src), ld_stream_v4(src + 8), g, sc, codes);
-      *reinterpret_cast<uint2*>(qx + m * (K / 2) + b * 8) = codes;
-    }
-    const int64_t r = m % 128;
-    sx[((m / 128) * steps + b / 4) * 512 + (r % 32) * 16 + (r / 32) * 4 + (b % 4)] = (uint8_t)sc;
-  }
-}
-
 // ----------------------------------------------- MXFP4 scales as NVFP4 scales
 //
 // The two formats share the nibble layout, so MXFP4 weights run on the NVFP4
@@ -417,35 +286,6 @@ cudaError_t launch_mx_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t 
   const int grid = grid_for(N * (K / 32), sms);
   mx_quantize_kernel<<<grid, 256, 0, stream>>>(w, N, K, ldw, q, s);
   return cudaGetLastError();
-}
-
-cudaError_t launch_quantize_x_mma(const uint16_t* X, int64_t ldx, int64_t M, int64_t K, float* amax, bool given,
-                                  uint8_t* qx, uint8_t* sx, cudaStream_t stream, int sms) {
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(256);
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int64_t ldx_ = ldx, M_ = M, K_ = K;
-  int parts = 0;
-  if (!given) {
-    const int64_t blocks = (M * (K / 8) + 255) / 256;
-    parts = (int)(blocks < kXAmaxParts ? blocks : kXAmaxParts);
-    cfg.gridDim = dim3(parts);
-    void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&amax};
-    cudaError_t e = cudaLaunchKernelExC(&cfg, (const void*)x_amax_partial_kernel, args);
-    if (e != cudaSuccess) return e;
-  }
-  int64_t Mpad = (M + 255) / 256 * 256;
-  const int64_t blocks = (Mpad * (K / 16) + 255) / 256;
-  const int64_t cap = (int64_t)sms * 16;
-  cfg.gridDim = dim3((unsigned)(blocks < cap ? blocks : cap));
-  void* args[] = {(void*)&X, (void*)&ldx_, (void*)&M_, (void*)&K_, (void*)&Mpad, (void*)&amax, (void*)&parts,
-                  (void*)&qx, (void*)&sx};
-  return cudaLaunchKernelExC(&cfg, (const void*)quantize_x_mma_kernel, args);
 }
 
 cudaError_t launch_mx_to_nvfp4(const uint8_t* q, const uint8_t* s_mx, int64_t N, int64_t K, uint8_t* s_nv,
