@@ -457,7 +457,7 @@ nvfp4_status nvfp4_w4a4_gemm(const uint8_t* qx, const uint8_t* sx, const float* 
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
   cudaError_t e = nvfp4::launch_gemm_w4a4(qx, sx, x_amax, q, s_mma, g, Y, ldy, M, N, K,
-                                          (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0, (cudaStream_t)stream);
+                                          (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0, (cudaStream_t)stream, sms);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "W4A4 GEMM launch");
 }
 

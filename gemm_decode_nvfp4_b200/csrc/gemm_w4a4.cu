@@ -28,6 +28,8 @@
 //     the stage's own TMEM columns, then the MMA into the [128 x 256] fp32
 //     accumulator; each stage is committed to its "empty" barrier;
 //   - warps 2..5: the epilogue, TMEM -> g * g_x -> BF16 Y through shared memory.
+// The kernel is persistent (one CTA per SM, tiles in a fixed stride), so
+// the next tile's stages stream in while the epilogue drains the accumulator.
 // A stage's TMEM scale columns are rewritten only after the MMAs that read
 // them have completed (the stage's empty barrier), and tcgen05.cp is ordered
 // before the MMAs its thread issues after it.  Every wait is bounded.
@@ -67,15 +69,21 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle)");
 static_assert(kSfCol0 + kStages * 4 * kSfColsPerMma <= kTmemCols, "TMEM columns");
 
+constexpr int kEpiWarps = 4;
+constexpr int kEpiBytes = kEpiWarps * 2048;  // each epilogue warp's 32 x 32 BF16 staging block
+
 struct Bars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t tmem_full;
+  uint64_t acc_full;   // the accumulator of the current tile is complete (one phase per tile)
+  uint64_t acc_empty;  // the epilogue has read it (kEpiWarps arrivals per tile)
+  uint64_t mma_done;   // every MMA of the CTA has finished (teardown)
   uint32_t tmem_addr;
   volatile int err;
 };
 
-constexpr int kSmemBytes = kStages * kStageBytes + (int)sizeof(Bars) + 1024;
+constexpr int kSmemBytes = kStages * kStageBytes + kEpiBytes + (int)sizeof(Bars) + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Bars* bars) {
   if (bars->err) return false;
@@ -119,6 +127,11 @@ __global__ void __launch_bounds__(256) scales_to_mma_kernel(const uint8_t* __res
   }
 }
 
+// Persistent: gridDim.x CTAs (at most one per SM) take the tiles
+// t = blockIdx.x, blockIdx.x + gridDim.x, ... (weight tile t % tiles_n, token
+// tile t / tiles_n).  The ring's stage counter runs on across tiles, so the
+// producer streams the next tile while the epilogue drains the accumulator;
+// the next tile's first MMA waits for the epilogue (acc_empty).
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                      const uint8_t* __restrict__ s_mma, const uint8_t* __restrict__ sx,
@@ -131,20 +144,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto b_tile = [&](int st) { return smem + st * kStageBytes + kABytes; };
   auto sfa = [&](int st) { return smem + st * kStageBytes + kABytes + kBBytes; };
   auto sfb = [&](int st) { return smem + st * kStageBytes + kABytes + kBBytes + kSFABytes; };
-  Bars* bars = reinterpret_cast<Bars*>(smem + kStages * kStageBytes);
+  uint8_t* epi = smem + kStages * kStageBytes;
+  Bars* bars = reinterpret_cast<Bars*>(epi + kEpiBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = blockIdx.x, mt = blockIdx.y;
-  const int n0 = nt * kBM, m0 = mt * kBN;
   const int steps64 = K / 64;
   const int num_ks = K / kStageK;
+  const int tiles_n = (N + kBM - 1) / kBM;
+  const int tiles = tiles_n * ((M + kBN - 1) / kBN);
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kStages; ++st) {
       ptx::mbar_init(&bars->full[st], 1);
       ptx::mbar_init(&bars->empty[st], 1);
     }
-    ptx::mbar_init(&bars->tmem_full, 1);
+    ptx::mbar_init(&bars->acc_full, 1);
+    ptx::mbar_init(&bars->acc_empty, kEpiWarps);
+    ptx::mbar_init(&bars->mma_done, 1);
     bars->err = 0;
     ptx::fence_mbar_init();
   }
@@ -165,82 +181,109 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      const uint8_t* sa_src = s_mma + (int64_t)nt * steps64 * 512;
-      const uint8_t* sb_src0 = sx + (int64_t)(2 * mt) * steps64 * 512;
-      const uint8_t* sb_src1 = sx + (int64_t)(2 * mt + 1) * steps64 * 512;
-      auto issue_w = [&](int ks) {
-        const int st = ks % kStages;
-        ptx::tma_load_2d(a_tile(st), &tmap_w, &bars->full[st], ks * 128, n0);
-        ptx::bulk_load(sfa(st), sa_src + ks * kSFABytes, kSFABytes, &bars->full[st]);
-      };
-      auto issue_x = [&](int ks) {
-        const int st = ks % kStages;
-        ptx::tma_load_2d(b_tile(st), &tmap_x, &bars->full[st], ks * 128, m0);
-        ptx::bulk_load(sfb(st), sb_src0 + ks * 2048, 2048, &bars->full[st]);
-        ptx::bulk_load(sfb(st) + 2048, sb_src1 + ks * 2048, 2048, &bars->full[st]);
-      };
-      // static weights: the first stages' weights stream before the producer
-      // of X has finished
-      const int first = num_ks < kStages ? num_ks : kStages;
-      for (int ks = 0; ks < first; ++ks) ptx::mbar_arrive_expect_tx(&bars->full[ks], kStageBytes);
-      if (static_weights)
-        for (int ks = 0; ks < first; ++ks) issue_w(ks);
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int ks = 0; ks < first; ++ks) {
-        if (!static_weights) issue_w(ks);
-        issue_x(ks);
-      }
-      int next = first;
-      for (; next < num_ks; ++next) {
-        const int st = next % kStages;
-        if (!wait_or_fail(&bars->empty[st], ((next / kStages) - 1) & 1, bars)) break;
-        ptx::mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
-        issue_w(next);
-        issue_x(next);
+      int gi = 0;  // stages issued so far (over all tiles of this CTA)
+      bool first = true;
+      for (int t = blockIdx.x; t < tiles && !bars->err; t += gridDim.x) {
+        const int nt = t % tiles_n, mt = t / tiles_n;
+        const int n0 = nt * kBM, m0 = mt * kBN;
+        const uint8_t* sa_src = s_mma + (int64_t)nt * steps64 * 512;
+        const uint8_t* sb_src0 = sx + (int64_t)(2 * mt) * steps64 * 512;
+        const uint8_t* sb_src1 = sx + (int64_t)(2 * mt + 1) * steps64 * 512;
+        auto issue_w = [&](int st, int ks) {
+          ptx::tma_load_2d(a_tile(st), &tmap_w, &bars->full[st], ks * 128, n0);
+          ptx::bulk_load(sfa(st), sa_src + ks * kSFABytes, kSFABytes, &bars->full[st]);
+        };
+        auto issue_x = [&](int st, int ks) {
+          ptx::tma_load_2d(b_tile(st), &tmap_x, &bars->full[st], ks * 128, m0);
+          ptx::bulk_load(sfb(st), sb_src0 + ks * 2048, 2048, &bars->full[st]);
+          ptx::bulk_load(sfb(st) + 2048, sb_src1 + ks * 2048, 2048, &bars->full[st]);
+        };
+        int ks = 0;
+        if (first) {
+          // the ring starts empty; with static weights the first stages'
+          // weights stream before the producer of X has finished
+          const int f = num_ks < kStages ? num_ks : kStages;
+          for (int k = 0; k < f; ++k) ptx::mbar_arrive_expect_tx(&bars->full[k], kStageBytes);
+          if (static_weights)
+            for (int k = 0; k < f; ++k) issue_w(k, k);
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          for (int k = 0; k < f; ++k) {
+            if (!static_weights) issue_w(k, k);
+            issue_x(k, k);
+          }
+          ks = f;
+          gi = f;
+          first = false;
+        }
+        for (; ks < num_ks; ++ks) {
+          const int st = gi % kStages;
+          if (gi >= kStages && !wait_or_fail(&bars->empty[st], ((gi / kStages) - 1) & 1, bars)) break;
+          ptx::mbar_arrive_expect_tx(&bars->full[st], kStageBytes);
+          issue_w(st, ks);
+          issue_x(st, ks);
+          ++gi;
+        }
       }
       if (bars->err) {
         // let the copies already issued land before the CTA exits
-        for (int ks = next > kStages ? next - kStages : 0; ks < next; ++ks)
-          ptx::mbar_wait(&bars->full[ks % kStages], (ks / kStages) & 1, kWaitLimitNs);
+        for (int j = gi > kStages ? gi - kStages : 0; j < gi; ++j)
+          ptx::mbar_wait(&bars->full[j % kStages], (j / kStages) & 1, kWaitLimitNs);
       }
     }
   } else if (warp == 1) {
     // --------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      for (int ks = 0; ks < num_ks; ++ks) {
-        const int st = ks % kStages;
-        if (!wait_or_fail(&bars->full[st], (ks / kStages) & 1, bars)) break;
-        ptx::tc_fence_after();
-        const uint32_t a0 = ptx::smem_u32(a_tile(st)), b0 = ptx::smem_u32(b_tile(st));
-        const uint32_t fa = ptx::smem_u32(sfa(st)), fb = ptx::smem_u32(sfb(st));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma;
-          ptx::tmem_copy_sf(col, ptx::rows16_desc(fa + kk * 512));
-          ptx::tmem_copy_sf(col + 4, ptx::rows16_desc(fb + kk * 512));
-          ptx::tmem_copy_sf(col + 8, ptx::rows16_desc(fb + 2048 + kk * 512));
-          ptx::mma_nvf4(tmem, ptx::sw128_kmajor_desc(a0 + 32 * kk), ptx::sw128_kmajor_desc(b0 + 32 * kk), kIdesc,
-                        col, col + 4, (ks | kk) != 0);
+      int gi = 0, it = 0;
+      for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+        // the accumulator is free once the epilogue has read the previous tile
+        if (it > 0) {
+          if (!wait_or_fail(&bars->acc_empty, (it - 1) & 1, bars)) break;
+          ptx::tc_fence_after();
         }
-        ptx::mma_commit(&bars->empty[st]);
+        bool ok = true;
+        for (int ks = 0; ks < num_ks; ++ks, ++gi) {
+          const int st = gi % kStages;
+          if (!wait_or_fail(&bars->full[st], (gi / kStages) & 1, bars)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(a_tile(st)), b0 = ptx::smem_u32(b_tile(st));
+          const uint32_t fa = ptx::smem_u32(sfa(st)), fb = ptx::smem_u32(sfb(st));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma;
+            ptx::tmem_copy_sf(col, ptx::rows16_desc(fa + kk * 512));
+            ptx::tmem_copy_sf(col + 4, ptx::rows16_desc(fb + kk * 512));
+            ptx::tmem_copy_sf(col + 8, ptx::rows16_desc(fb + 2048 + kk * 512));
+            ptx::mma_nvf4(tmem, ptx::sw128_kmajor_desc(a0 + 32 * kk), ptx::sw128_kmajor_desc(b0 + 32 * kk),
+                          kIdesc, col, col + 4, (ks | kk) != 0);
+          }
+          ptx::mma_commit(&bars->empty[st]);
+        }
+        if (!ok) break;
+        ptx::mma_commit(&bars->acc_full);
       }
-      // arrives when every MMA above is done (also on the error path, so that
-      // TMEM is never freed under a running MMA)
-      ptx::mma_commit(&bars->tmem_full);
-      if (bars->err) ptx::mbar_wait(&bars->tmem_full, 0, kWaitLimitNs);
+      // arrives when every MMA above is done, so that TMEM is never freed
+      // under a running MMA (also on the error path)
+      ptx::mma_commit(&bars->mma_done);
+      ptx::mbar_wait(&bars->mma_done, 0, kWaitLimitNs);
     }
   } else {
     // ----------------------------------------------------------------- epilogue
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x_amax and Y
-    const bool acc_ready = __all_sync(0xFFFFFFFFu, wait_or_fail(&bars->tmem_full, 0, bars));
-    if (acc_ready) {
+    const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. +31 = weight rows of the tile
+    const float scale = __fmul_rn(*g, __fdiv_rn(*x_amax, 2688.0f));
+    // each 32 x 32 block (weight rows of this quarter x tokens) goes through
+    // this warp's 2 KB so that Y is written as 64-byte runs
+    const uint32_t stage = ptx::smem_u32(epi) + (uint32_t)(warp - kEpiWarp0) * 2048u;
+    const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+    int it = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+      const int nt = t % tiles_n, mt = t / tiles_n;
+      const int n0 = nt * kBM, m0 = mt * kBN;
+      if (!__all_sync(0xFFFFFFFFu, wait_or_fail(&bars->acc_full, it & 1, bars))) break;
       ptx::tc_fence_after();
-      const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. +31 = weight rows
-      const float scale = __fmul_rn(*g, __fdiv_rn(*x_amax, 2688.0f));
-      // each 32 x 32 block (weight rows of this quarter x tokens) goes through
-      // 2 KB of the idle stage-0 buffers so that Y is written as 64-byte runs
-      const uint32_t stage = ptx::smem_u32(a_tile(0)) + (uint32_t)(warp - kEpiWarp0) * 2048u;
-      const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
 #pragma unroll 1
       for (int c0 = 0; c0 < kBN && m0 + c0 < M; c0 += 32) {
         uint32_t rr[32];
@@ -270,6 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
+      // every TMEM read of this tile has completed (tcgen05.wait::ld above)
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->acc_empty);
     }
   }
 
@@ -412,7 +459,7 @@ cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t
 
 cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
                              const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
-                             int64_t K, bool static_weights, cudaStream_t stream) {
+                             int64_t K, bool static_weights, cudaStream_t stream, int sms) {
   CUtensorMap tw, tx;
   if (!tc::make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
                         128u, (uint32_t)kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -430,8 +477,9 @@ cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* 
   }
   int m = (int)M, n = (int)N, k = (int)K, sw = static_weights ? 1 : 0;
   void* args[] = {&tw, &tx, (void*)&s_mma, (void*)&sx, (void*)&g, (void*)&x_amax, &Y, &ldy, &m, &n, &k, &sw};
-  dim3 grid((unsigned)((N + kBM - 1) / kBM), (unsigned)((M + kBN - 1) / kBN));
-  return tc::launch_pdl((const void*)gemm_w4a4_kernel, grid, dim3(kThreads), kSmemBytes, stream, args);
+  const int64_t tiles = (N + kBM - 1) / kBM * ((M + kBN - 1) / kBN);
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // one persistent CTA per SM at most
+  return tc::launch_pdl((const void*)gemm_w4a4_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, args);
 }
 
 cudaError_t read_and_clear_w4a4_timeouts(unsigned int* count) {
