@@ -376,6 +376,9 @@ nvfp4_status check_w4a4_shape(int64_t M, int64_t N, int64_t K) {
   if (M < 0 || N < 0) return fail(NVFP4_ERR_SHAPE, "negative size M=%lld N=%lld", (long long)M, (long long)N);
   if (M > ((int64_t)1 << 24) || N > ((int64_t)1 << 31) - 128)
     return fail(NVFP4_ERR_SHAPE, "M=%lld or N=%lld too large", (long long)M, (long long)N);
+  // the GEMM numbers its 128 x 256 output tiles with 32-bit integers
+  if ((N + 127) / 128 * ((M + 255) / 256) > (int64_t)INT32_MAX)
+    return fail(NVFP4_ERR_SHAPE, "M=%lld x N=%lld has too many 128 x 256 tiles", (long long)M, (long long)N);
   return NVFP4_OK;
 }
 

@@ -28,7 +28,8 @@
  *       (nvfp4_w4a4_x_scales_bytes).
  *   Y   BF16 [M, N], leading dimension ldy
  *
- * K must be a positive multiple of 256 and at most 2^24; N >= 1; 1 <= M <= 2^24.
+ * K must be a positive multiple of 256 and at most 2^24; N >= 1; 1 <= M <= 2^24;
+ * ceil(N / 128) * ceil(M / 256) < 2^31 (the GEMM's tile count).
  * X, q, qx, scale buffers and the workspace are 16-byte aligned, ldx a
  * multiple of 8; g and x_amax 4-byte aligned; Y 2-byte aligned.
  */

@@ -156,3 +156,12 @@ def test_w4a4_binding_constants_match_header():
         text = f.read()
     assert int(re.search(r"#define NVFP4_W4A4_AMAX_FLOATS (\d+)", text).group(1)) == nv.AMAX_FLOATS
     assert int(re.search(r"#define NVFP4_W4A4_GIVEN_AMAX (\d+)u", text).group(1)) == nv.GIVEN_AMAX
+
+
+def test_w4a4_tile_count_bound():
+    """2^24 tokens x 2^31 - 128 weight rows is within the per-dimension limits
+    but has more 128 x 256 tiles than a 32-bit tile index holds."""
+    L = nv.lib
+    big_n = (1 << 31) - 128
+    assert L.nvfp4_w4a4_gemm(A, A, A, A, A, A, A, big_n, 1 << 24, big_n, 256, 0, None) == SHAPE
+    assert b"tiles" in L.nvfp4_last_error()
