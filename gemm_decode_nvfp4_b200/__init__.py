@@ -382,12 +382,35 @@ def w4a4_quantize_x(X: torch.Tensor, x_amax: torch.Tensor, given_amax: bool = Fa
     return qx, sx
 
 
+def _need_w4a4_weights(q: torch.Tensor, s_mma: torch.Tensor, g: torch.Tensor):
+    """q [N, K/2] contiguous, s_mma holding the rearranged scales of [N, K/16]
+    (w4a4_prepare_weights), g an fp32 tensor scale.  Returns (N, K)."""
+    _need(q, torch.uint8, "q", 2)
+    _need(s_mma, torch.uint8, "s_mma")
+    _need(g, torch.float32, "g")
+    if not q.is_contiguous() or not s_mma.is_contiguous():
+        raise ValueError("q and s_mma must be contiguous")
+    N, K = q.shape[0], q.shape[1] * 2
+    if s_mma.numel() < lib.nvfp4_w4a4_weight_scales_bytes(N, K):
+        raise ValueError(f"s_mma holds {s_mma.numel()} bytes, [{N}, {K}] needs "
+                         f"{lib.nvfp4_w4a4_weight_scales_bytes(N, K)} (w4a4_prepare_weights)")
+    return N, K
+
+
 def w4a4_gemm(qx, sx, x_amax, q, s_mma, g, Y, stream=None, static_weights: bool = False) -> None:
+    """Y [M, N] = bf16(g * (x_amax[0] / 2688) * Xq . Wq^T) from quantized
+    activations (qx, sx, x_amax from w4a4_quantize_x) and weights (q, s_mma
+    from w4a4_prepare_weights, g)."""
     _need(Y, torch.bfloat16, "Y", 2)
-    M, N = Y.shape
-    K = q.shape[1] * 2
-    if qx.shape != (M, K // 2) or q.shape[0] != N:
+    _need(qx, torch.uint8, "qx", 2)
+    _need(sx, torch.uint8, "sx")
+    _need(x_amax, torch.float32, "x_amax")
+    N, K = _need_w4a4_weights(q, s_mma, g)
+    M = Y.shape[0]
+    if qx.shape != (M, K // 2) or Y.shape[1] != N or not qx.is_contiguous() or not sx.is_contiguous():
         raise ValueError(f"shape mismatch: qx {tuple(qx.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
+    if sx.numel() < lib.nvfp4_w4a4_x_scales_bytes(M, K):
+        raise ValueError(f"sx holds {sx.numel()} bytes, [{M}, {K}] needs {lib.nvfp4_w4a4_x_scales_bytes(M, K)}")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
     _check("nvfp4_w4a4_gemm", lib.nvfp4_w4a4_gemm(_ptr(qx), _ptr(sx), _ptr(x_amax), _ptr(q), _ptr(s_mma), _ptr(g),
                                                    _ptr(Y), Y.stride(0), M, N, K, flags, _stream(stream)))
@@ -405,9 +428,11 @@ def w4a4_linear(X: torch.Tensor, q: torch.Tensor, s_mma: torch.Tensor, g: torch.
     _need(X, torch.bfloat16, "X", 2)
     _need(Y, torch.bfloat16, "Y", 2)
     _need(workspace, torch.uint8, "workspace")
+    if x_amax is not None:
+        _need(x_amax, torch.float32, "x_amax")
+    N, Kq = _need_w4a4_weights(q, s_mma, g)
     M, K = X.shape
-    N = q.shape[0]
-    if q.shape[1] * 2 != K or Y.shape != (M, N):
+    if Kq != K or Y.shape != (M, N):
         raise ValueError(f"shape mismatch: X {tuple(X.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
     if X.stride(1) != 1:
