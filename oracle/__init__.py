@@ -56,6 +56,8 @@ def lib():
         L.oracle_tensor_scale.restype = c_f
         L.oracle_quantize.argtypes = [c_p, c_i64, c_i64, c_i64, c_f, c_p, c_p]
         L.oracle_quantize.restype = None
+        L.oracle_quantize_mse.argtypes = [c_p, c_i64, c_i64, c_i64, c_f, ctypes.c_int, c_p, c_p]
+        L.oracle_quantize_mse.restype = None
         L.oracle_dequantize.argtypes = [c_p, c_p, c_f, c_i64, c_i64, c_p]
         L.oracle_dequantize.restype = None
         L.oracle_linear.argtypes = [c_p, c_i64, c_p, c_p, c_f, c_i64, c_i64, c_i64,
@@ -142,6 +144,24 @@ def quantize(w, g=None):
     q = np.empty((N, K // 2), np.uint8)
     s = np.empty((N, K // 16), np.uint8)
     lib().oracle_quantize(_ptr(b), N, K, K, float(g), _ptr(q), _ptr(s))
+    return q, s, g
+
+
+def quantize_mse(w, g=None, window: int = 8):
+    """NVFP4 with each micro-scale chosen by the least squared reconstruction
+    error over the E4M3 codes within `window` codes of the round-to-nearest
+    one (imp docs/quantization.md, micro-scale search paragraph; readings in
+    nvfp4_oracle.c).  Returns (q, s, g) like quantize; window 0 is quantize."""
+    b = _bf16_bits(w)
+    N, K = b.shape
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    if g is None:
+        g = tensor_scale(amax(b))
+    g = np.float32(g)
+    q = np.empty((N, K // 2), np.uint8)
+    s = np.empty((N, K // 16), np.uint8)
+    lib().oracle_quantize_mse(_ptr(b), N, K, K, float(g), int(window), _ptr(q), _ptr(s))
     return q, s, g
 
 
