@@ -226,13 +226,14 @@ NVFP4_API nvfp4_status nvfp4_gemv_grouped(const uint16_t* X, int64_t ldx, const 
                                           int64_t K, uint32_t flags, nvfp4_stream_t stream);
 
 /*
- * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMMs
- * and the TMA-fed decode GEMV) is bounded (about 2 s); a CTA that gives up
- * records it in a device counter and finishes without hanging, leaving its
- * outputs undefined.  This call reads and
- * clears that counter for the current device (it waits for prior work on the
- * legacy default stream) and returns NVFP4_ERR_TIMEOUT if it was non-zero,
- * else NVFP4_ERR_INVALID_ARG if grouped GEMVs met out-of-range ids.
+ * Diagnostic: every wait inside the pipelined kernels (the tensor-core GEMMs,
+ * the W4A4 GEMM of nvfp4_w4a4.h and the TMA-fed decode GEMV) is bounded
+ * (about 2 s); a CTA that gives up records it in a device counter and finishes
+ * without hanging, leaving its outputs undefined.  This call reads and clears
+ * those counters for the current device (it waits for prior work on the
+ * legacy default stream) and returns NVFP4_ERR_TIMEOUT if one was non-zero,
+ * else NVFP4_ERR_INVALID_ARG if grouped GEMVs met out-of-range ids or MXFP4
+ * scales could not be restated (mxfp4.h, mxfp4_to_nvfp4_scales).
  */
 NVFP4_API nvfp4_status nvfp4_check_device_errors(void);
 
