@@ -165,3 +165,16 @@ def test_w4a4_tile_count_bound():
     big_n = (1 << 31) - 128
     assert L.nvfp4_w4a4_gemm(A, A, A, A, A, A, A, big_n, 1 << 24, big_n, 256, 0, None) == SHAPE
     assert b"tiles" in L.nvfp4_last_error()
+
+
+def test_mxfp4_to_nvfp4_scales_validation():
+    L = nv.lib
+    assert "mxfp4_to_nvfp4_scales" in nv.declared_symbols()
+    for K in (0, 48, -32):
+        assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, K, A + 8192, A + 12288, None) == SHAPE
+    assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 0, 64, A + 8192, A + 12288, None) == OK      # no-op
+    assert L.mxfp4_to_nvfp4_scales(None, A + 4096, 4, 64, A + 8192, A + 12288, None) == INVALID
+    assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 8200, A + 12288, None) == ALIGN   # s_nv
+    assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 8192, A + 12290, None) == ALIGN   # g_out
+    assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 64, A + 12288, None) == INVALID   # s_nv in q
+    assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 8192, A + 4100, None) == INVALID  # g_out in s_mx
