@@ -104,9 +104,28 @@ def declared_symbols() -> list[str]:
     return names
 
 
-def _stream(stream=None) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _device(*tensors) -> torch.device:
+    """The one CUDA device all the given tensors (None skipped) live on."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"tensors must all be on one CUDA device, got {sorted(str(d) for d in devs)}")
+    return devs.pop()
+
+
+def _stream(stream, dev: torch.device) -> int:
+    """The raw stream handle for a call on `dev`: the given stream (which must
+    belong to `dev`) or that device's current stream."""
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    if s.device != dev:
+        raise ValueError(f"stream is on {s.device}, the tensors on {dev}")
     return s.cuda_stream
+
+
+def _call(fn: str, dev: torch.device, *args) -> None:
+    """Call lib.<fn>(*args) with `dev` current (the library launches on the
+    current device) and raise on a non-zero status."""
+    with torch.cuda.device(dev):
+        _check(fn, getattr(lib, fn)(*args))
 
 
 def _ptr(t: torch.Tensor | None):
@@ -133,8 +152,8 @@ def amax(w: torch.Tensor, out: torch.Tensor, stream=None) -> None:
     _need(w, torch.bfloat16, "w")
     _need(out, torch.float32, "out")
     w2 = w if w.dim() == 2 else w.reshape(1, -1)
-    _check("nvfp4_amax", lib.nvfp4_amax(_ptr(w2), w2.shape[0], w2.shape[1], w2.stride(0),
-                                        _ptr(out), _stream(stream)))
+    dev = _device(w, out)
+    _call("nvfp4_amax", dev, _ptr(w2), w2.shape[0], w2.shape[1], w2.stride(0), _ptr(out), _stream(stream, dev))
 
 
 def quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch.Tensor | None,
@@ -151,8 +170,9 @@ def quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch.Ten
         _need(g_out, torch.float32, "g_out")
     if amax is not None:
         _need(amax, torch.float32, "amax")
-    _check("nvfp4_quantize", lib.nvfp4_quantize(_ptr(w), N, K, w.stride(0), _ptr(amax), _ptr(q), _ptr(s),
-                                                _ptr(g_out), _stream(stream)))
+    dev = _device(w, q, s, g_out, amax)
+    _call("nvfp4_quantize", dev, _ptr(w), N, K, w.stride(0), _ptr(amax), _ptr(q), _ptr(s), _ptr(g_out),
+          _stream(stream, dev))
 
 
 FLAG_STATIC_WEIGHTS = 1
@@ -173,8 +193,8 @@ def gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, y: 
     if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
-    _check("nvfp4_gemv_ex", lib.nvfp4_gemv_ex(_ptr(x), _ptr(q), _ptr(s), _ptr(g), _ptr(y), N, K, flags,
-                                              _stream(stream)))
+    dev = _device(x, q, s, g, y)
+    _call("nvfp4_gemv_ex", dev, _ptr(x), _ptr(q), _ptr(s), _ptr(g), _ptr(y), N, K, flags, _stream(stream, dev))
 
 
 def gemm_workspace_size(M: int, N: int, K: int) -> int:
@@ -200,8 +220,9 @@ def gemm(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, Y: 
         _need(workspace, torch.uint8, "workspace")
         ws_bytes = workspace.numel()
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
-    _check("nvfp4_gemm_ex", lib.nvfp4_gemm_ex(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0),
-                                              M, N, K, _ptr(workspace), ws_bytes, flags, _stream(stream)))
+    dev = _device(X, q, s, g, Y, workspace)
+    _call("nvfp4_gemm_ex", dev, _ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0), M, N, K,
+          _ptr(workspace), ws_bytes, flags, _stream(stream, dev))
 
 
 def _header_constant(name: str) -> int:
@@ -233,8 +254,9 @@ def gemm_noalloc(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Ten
     if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
-    _check("nvfp4_gemm_noalloc", lib.nvfp4_gemm_noalloc(_ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y),
-                                                        Y.stride(0), M, N, K, flags, _stream(stream)))
+    dev = _device(X, q, s, g, Y)  # the built-in scratch of this device is used
+    _call("nvfp4_gemm_noalloc", dev, _ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(Y), Y.stride(0), M, N,
+          K, flags, _stream(stream, dev))
 
 
 # ------------------------------------------------------ allocating helpers
@@ -273,7 +295,8 @@ def mx_quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, stream=None) 
         raise ValueError("w rows and q, s must be contiguous")
     if q.shape != (N, K // 2) or s.shape != (N, K // 32):
         raise ValueError("q/s must be [N, K/2] / [N, K/32]")
-    _check("mxfp4_quantize", lib.mxfp4_quantize(_ptr(w), N, K, w.stride(0), _ptr(q), _ptr(s), _stream(stream)))
+    dev = _device(w, q, s)
+    _call("mxfp4_quantize", dev, _ptr(w), N, K, w.stride(0), _ptr(q), _ptr(s), _stream(stream, dev))
 
 
 def mx_quantize_new(w: torch.Tensor, stream=None):
@@ -298,7 +321,8 @@ def mx_gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, y: torch.Tensor, 
     if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 32):
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/32]")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
-    _check("mxfp4_gemv_ex", lib.mxfp4_gemv_ex(_ptr(x), _ptr(q), _ptr(s), _ptr(y), N, K, flags, _stream(stream)))
+    dev = _device(x, q, s, y)
+    _call("mxfp4_gemv_ex", dev, _ptr(x), _ptr(q), _ptr(s), _ptr(y), N, K, flags, _stream(stream, dev))
 
 
 # ------------------------------------------------------------ grouped (MoE) GEMV
@@ -323,9 +347,10 @@ def gemv_grouped(X: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Ten
         raise ValueError("q/s/g must be contiguous [E, N, K/2] / [E, N, K/16] / [E]")
     if token_ids.numel() != P or not expert_ids.is_contiguous() or not token_ids.is_contiguous():
         raise ValueError("expert_ids and token_ids must be contiguous [P]")
-    _check("nvfp4_gemv_grouped", lib.nvfp4_gemv_grouped(
-        _ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(expert_ids), _ptr(token_ids), _ptr(Y), Y.stride(0),
-        P, E, T, N, K, 0, _stream(stream)))
+    dev = _device(X, q, s, g, expert_ids, token_ids, Y)
+    _call("nvfp4_gemv_grouped", dev,
+          _ptr(X), X.stride(0), _ptr(q), _ptr(s), _ptr(g), _ptr(expert_ids), _ptr(token_ids), _ptr(Y), Y.stride(0),
+          P, E, T, N, K, 0, _stream(stream, dev))
 
 
 def mx_to_nvfp4(q: torch.Tensor, s_mx: torch.Tensor, stream=None):
@@ -339,8 +364,8 @@ def mx_to_nvfp4(q: torch.Tensor, s_mx: torch.Tensor, stream=None):
         raise ValueError("q/s_mx must be contiguous [N, K/2] / [N, K/32]")
     s_nv = torch.empty((N, K // 16), dtype=torch.uint8, device=q.device)
     g = torch.empty((1,), dtype=torch.float32, device=q.device)
-    _check("mxfp4_to_nvfp4_scales", lib.mxfp4_to_nvfp4_scales(_ptr(q), _ptr(s_mx), N, K, _ptr(s_nv), _ptr(g),
-                                                               _stream(stream)))
+    dev = _device(q, s_mx)
+    _call("mxfp4_to_nvfp4_scales", dev, _ptr(q), _ptr(s_mx), N, K, _ptr(s_nv), _ptr(g), _stream(stream, dev))
     return s_nv, g
 
 
@@ -359,7 +384,8 @@ def w4a4_prepare_weights(s: torch.Tensor, K: int, stream=None) -> torch.Tensor:
     if not s.is_contiguous() or s.shape[1] * 16 != K:
         raise ValueError("s must be contiguous [N, K/16]")
     out = torch.empty((lib.nvfp4_w4a4_weight_scales_bytes(N, K),), dtype=torch.uint8, device=s.device)
-    _check("nvfp4_w4a4_prepare_weights", lib.nvfp4_w4a4_prepare_weights(_ptr(s), N, K, _ptr(out), _stream(stream)))
+    dev = _device(s)
+    _call("nvfp4_w4a4_prepare_weights", dev, _ptr(s), N, K, _ptr(out), _stream(stream, dev))
     return out
 
 
@@ -377,8 +403,9 @@ def w4a4_quantize_x(X: torch.Tensor, x_amax: torch.Tensor, given_amax: bool = Fa
     ldx = X.stride(0)
     qx = torch.empty((M, K // 2), dtype=torch.uint8, device=X.device)
     sx = torch.empty((lib.nvfp4_w4a4_x_scales_bytes(M, K),), dtype=torch.uint8, device=X.device)
-    _check("nvfp4_w4a4_quantize_x", lib.nvfp4_w4a4_quantize_x(_ptr(X), ldx, M, K, _ptr(qx), _ptr(sx), _ptr(x_amax),
-                                                               GIVEN_AMAX if given_amax else 0, _stream(stream)))
+    dev = _device(X, x_amax)
+    _call("nvfp4_w4a4_quantize_x", dev, _ptr(X), ldx, M, K, _ptr(qx), _ptr(sx), _ptr(x_amax),
+          GIVEN_AMAX if given_amax else 0, _stream(stream, dev))
     return qx, sx
 
 
@@ -412,8 +439,9 @@ def w4a4_gemm(qx, sx, x_amax, q, s_mma, g, Y, stream=None, static_weights: bool 
     if sx.numel() < lib.nvfp4_w4a4_x_scales_bytes(M, K):
         raise ValueError(f"sx holds {sx.numel()} bytes, [{M}, {K}] needs {lib.nvfp4_w4a4_x_scales_bytes(M, K)}")
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
-    _check("nvfp4_w4a4_gemm", lib.nvfp4_w4a4_gemm(_ptr(qx), _ptr(sx), _ptr(x_amax), _ptr(q), _ptr(s_mma), _ptr(g),
-                                                   _ptr(Y), Y.stride(0), M, N, K, flags, _stream(stream)))
+    dev = _device(qx, sx, x_amax, q, s_mma, g, Y)
+    _call("nvfp4_w4a4_gemm", dev, _ptr(qx), _ptr(sx), _ptr(x_amax), _ptr(q), _ptr(s_mma), _ptr(g), _ptr(Y),
+          Y.stride(0), M, N, K, flags, _stream(stream, dev))
 
 
 def w4a4_workspace_size(M: int, K: int) -> int:
@@ -437,6 +465,6 @@ def w4a4_linear(X: torch.Tensor, q: torch.Tensor, s_mma: torch.Tensor, g: torch.
     flags = FLAG_STATIC_WEIGHTS if static_weights else 0
     if X.stride(1) != 1:
         raise ValueError("X rows must be contiguous")
-    _check("nvfp4_w4a4_linear", lib.nvfp4_w4a4_linear(_ptr(X), X.stride(0), _ptr(x_amax), _ptr(q), _ptr(s_mma),
-                                                       _ptr(g), _ptr(Y), Y.stride(0), M, N, K, _ptr(workspace),
-                                                       workspace.numel(), flags, _stream(stream)))
+    dev = _device(X, x_amax, q, s_mma, g, Y, workspace)
+    _call("nvfp4_w4a4_linear", dev, _ptr(X), X.stride(0), _ptr(x_amax), _ptr(q), _ptr(s_mma), _ptr(g), _ptr(Y),
+          Y.stride(0), M, N, K, _ptr(workspace), workspace.numel(), flags, _stream(stream, dev))

@@ -19,21 +19,25 @@
 // between them, or host threads racing on one device) use the same bytes and
 // race; calls must be ordered, e.g. issued on one stream.
 //
-// Set-up: the first call on each device, with that device current, looks up
-// the array's device address with cudaGetSymbolAddress (the host-side name of
-// a __device__ array is not a device address) and caches it.  Make that first
-// call before any stream capture on the device begins.  Nothing here calls
-// cudaMalloc, cudaFree or any other allocating routine.
-#include <atomic>
+// Set-up: the first call in each CUDA context (normally a device's primary
+// context), with that context current, looks up the array's device address
+// with cudaGetSymbolAddress (the host-side name of a __device__ array is not a
+// device address) and caches it under the context's unique id.  A later call
+// in another context (after cudaDeviceReset, or when the caller made a
+// different context current) looks it up again instead of reusing an address
+// of a context that may be gone.  Make the first call in a context before any
+// stream capture in it begins.  Nothing here calls cudaMalloc, cudaFree or any
+// other allocating routine.
 #include <mutex>
 
 #include "nvfp4.h"
 #include "nvfp4_kernels.h"
+#include "tc_host.h"
 
 namespace {
 
 constexpr size_t kScratchBytes = NVFP4_GEMM_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 }  // namespace
 
@@ -42,28 +46,36 @@ static __device__ __align__(256) unsigned char g_gemm_scratch[kScratchBytes];
 
 namespace {
 
+// Address of g_gemm_scratch per context id; a context's entry is replaced when
+// its slot is reused after kMaxContexts others.
+struct ScratchSlot {
+  unsigned long long ctx;
+  void* ptr;
+};
 std::mutex g_setup_mutex;
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
+ScratchSlot g_slots[kMaxContexts];
+int g_used = 0, g_next = 0;
 
-// Device address of g_gemm_scratch on the current device (set up once).
-nvfp4_status scratch_for_current_device(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return nvfp4::report_cuda_error(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return nvfp4::report_error(NVFP4_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
-    if (!p) {
-      e = cudaGetSymbolAddress(&p, g_gemm_scratch);
-      if (e != cudaSuccess || !p) {
-        return nvfp4::report_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
-                                        "cudaGetSymbolAddress of the built-in GEMM scratch");
-      }
-      g_scratch_ptr[dev].store(p, std::memory_order_release);
+// Device address of g_gemm_scratch in the context current on this thread.
+nvfp4_status scratch_for_current_context(void** out) {
+  unsigned long long ctx = 0;
+  cudaError_t e = nvfp4::tc::current_context_id(&ctx);
+  if (e != cudaSuccess) return nvfp4::report_cuda_error(e, "reading the current CUDA context");
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  for (int i = 0; i < g_used; ++i)
+    if (ctx != 0 && g_slots[i].ctx == ctx) {
+      *out = g_slots[i].ptr;
+      return NVFP4_OK;
     }
-  }
+  // (with no context current yet, this creates the device's primary context)
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_gemm_scratch);
+  if (e != cudaSuccess || !p)
+    return nvfp4::report_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                                    "cudaGetSymbolAddress of the built-in GEMM scratch");
+  if (ctx == 0 && (e = nvfp4::tc::current_context_id(&ctx)) != cudaSuccess)
+    return nvfp4::report_cuda_error(e, "reading the current CUDA context");
+  g_slots[g_used < kMaxContexts ? g_used++ : (g_next++ % kMaxContexts)] = {ctx, p};
   *out = p;
   return NVFP4_OK;
 }
@@ -73,6 +85,11 @@ nvfp4_status scratch_for_current_device(void** out) {
 NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,
                                            const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                                            uint32_t flags, nvfp4_stream_t stream) {
+  // the shape checks of nvfp4_gemm_ex, first, so that a bad shape gets the same status here
+  if (K <= 0 || K % 16 != 0)
+    return nvfp4::report_error(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 16", (long long)K);
+  if (M < 0 || N < 0)
+    return nvfp4::report_error(NVFP4_ERR_SHAPE, "negative size M=%lld N=%lld", (long long)M, (long long)N);
   const size_t need = nvfp4_gemm_workspace_size(M, N, K);
   if (need > kScratchBytes) {
     return nvfp4::report_error(NVFP4_ERR_WORKSPACE,
@@ -82,7 +99,7 @@ NVFP4_API nvfp4_status nvfp4_gemm_noalloc(const uint16_t* X, int64_t ldx, const 
                                (long long)M, (long long)K, need, kScratchBytes);
   }
   void* scratch = nullptr;
-  const nvfp4_status st = scratch_for_current_device(&scratch);
+  const nvfp4_status st = scratch_for_current_context(&scratch);
   if (st != NVFP4_OK) return st;
   return nvfp4_gemm_ex(X, ldx, q, s, g, Y, ldy, M, N, K, scratch, kScratchBytes, flags, stream);
 }

@@ -562,15 +562,9 @@ cudaError_t launch_small(const uint16_t* X, int64_t ldx, const uint16_t* Xh, con
                           (uint32_t)kBK, (uint32_t)BNT, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static tc::SmemOptIn opt_in;
+  const cudaError_t e = opt_in.ensure((const void*)gemm_small_kernel<BNT, CONV>, C::kSmem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(gemm_small_kernel<BNT, CONV>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
   int sw = static_weights ? 1 : 0;
   void* args[] = {&tw, &ts, &tx, (void*)&q, (void*)&s, (void*)&g, (void*)&info, (void*)&X, &ldx, &Y, &ldy,
                   &M, &N, &K, &sw};

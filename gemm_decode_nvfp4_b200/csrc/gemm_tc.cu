@@ -43,6 +43,7 @@
 #include "nvfp4_device.cuh"
 #include "nvfp4_kernels.h"
 #include "sm100_ptx.cuh"
+#include "tc_host.h"
 
 namespace nvfp4 {
 
@@ -548,38 +549,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-cudaError_t launch_pdl(const void* func, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelExC(&cfg, func, args);
-}
-
 template <int BN, int NSUB>
 cudaError_t launch_cfg(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,
                        uint16_t* Y, int64_t ldy, int M, int N, int K, const int* info, const uint16_t* Xh,
                        bool static_weights, cudaStream_t stream) {
   using C = Cfg<BN, NSUB>;
-  auto enc = encode_fn();
+  auto enc = tc::encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap tx, tw, ts;
   {
@@ -612,20 +587,14 @@ cudaError_t launch_cfg(const uint16_t* X, int64_t ldx, const uint8_t* q, const u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  static bool attr_set[64] = {};  // per device ordinal
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static tc::SmemOptIn opt_in;
+  const cudaError_t e = opt_in.ensure((const void*)gemm_tc_kernel<BN, NSUB>, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(gemm_tc_kernel<BN, NSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
   int sw = static_weights ? 1 : 0;
   void* args[] = {&tx, &tw, &ts, (void*)&q, (void*)&s, (void*)&g, (void*)&info, (void*)&X, &ldx, &Y, &ldy,
                   &M, &N, &K, &sw};
   dim3 grid((N + kBM - 1) / kBM, (M + C::kBNT - 1) / C::kBNT);
-  return launch_pdl((const void*)gemm_tc_kernel<BN, NSUB>, grid, dim3(kThreads), C::kSmemBytes, stream, args);
+  return tc::launch_pdl((const void*)gemm_tc_kernel<BN, NSUB>, grid, dim3(kThreads), C::kSmemBytes, stream, args);
 }
 
 size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
@@ -650,7 +619,7 @@ cudaError_t launch_gemm_prep(const uint16_t* X, int64_t ldx, int64_t M, int64_t 
   const uint16_t* xp = X;
   int kk = (int)K;
   void* args[] = {(void*)&xp, &ldx, &kk, (void*)&info, (void*)&Xh};
-  return launch_pdl((const void*)prep_x_kernel, dim3((unsigned)M), dim3(kPrepThreads), 0, stream, args);
+  return tc::launch_pdl((const void*)prep_x_kernel, dim3((unsigned)M), dim3(kPrepThreads), 0, stream, args);
 }
 
 cudaError_t launch_gemm_tc(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s, const float* g,

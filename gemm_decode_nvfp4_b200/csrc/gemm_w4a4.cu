@@ -466,15 +466,9 @@ cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* 
       !tc::make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, (uint64_t)(K / 2), (uint64_t)M, (uint64_t)(K / 2),
                         128u, (uint32_t)kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  static bool attr_set[64] = {};  // per device ordinal
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static tc::SmemOptIn opt_in;
+  const cudaError_t e = opt_in.ensure((const void*)gemm_w4a4_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
   int m = (int)M, n = (int)N, k = (int)K, sw = static_weights ? 1 : 0;
   void* args[] = {&tw, &tx, (void*)&s_mma, (void*)&sx, (void*)&g, (void*)&x_amax, &Y, &ldy, &m, &n, &k, &sw};
   const int64_t tiles = (N + kBM - 1) / kBM * ((M + kBN - 1) / kBN);

@@ -395,15 +395,9 @@ cudaError_t launch(const uint16_t* x, const uint8_t* q, const uint8_t* s, const 
                    int K, bool static_weights, cudaStream_t stream, const Problems& P, int num_problems) {
   const size_t smem = (size_t)K * sizeof(uint16_t);
   auto kern = gemv_kernel<R, CB, MINB, MX, GROUPED>;
-  static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static tc::SmemOptIn opt_in;
+  const cudaError_t e = opt_in.ensure((const void*)kern, (int)smem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || smem_set[dev] < (int)smem) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) smem_set[dev] = (int)smem;
-  }
   const int rows_per_cta = kWarps * R;
   const int grid = (N + rows_per_cta - 1) / rows_per_cta;
   cudaLaunchConfig_t cfg = {};
@@ -730,15 +724,9 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
              tc::make_tmap_3d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, sbytes, N, E, sbytes, N * sbytes,
                               MX ? kRingBK / 16 : kRingBK / 8, p.BR, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!*encoded) return cudaSuccess;
-  static int smem_set[64] = {};  // per device: largest dynamic shared memory enabled so far
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static tc::SmemOptIn opt_in;
+  const cudaError_t e = opt_in.ensure((const void*)gemv_ring_kernel<MX, GROUPED>, (int)p.smem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || smem_set[dev] < (int)p.smem) {
-    e = cudaFuncSetAttribute(gemv_ring_kernel<MX, GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) smem_set[dev] = (int)p.smem;
-  }
   int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S;
   Problems Pc = P;
   void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S, &Pc};

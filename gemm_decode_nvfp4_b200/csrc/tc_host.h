@@ -1,6 +1,7 @@
-// tc_host.h -- host-side helpers shared by the tensor-core launchers: TMA
-// tensor-map encoding (through the driver entry point, no libcuda link) and
-// kernel launch with programmatic dependent launch enabled.
+// tc_host.h -- host-side helpers shared by the kernel launchers: TMA
+// tensor-map encoding (through the driver entry point, no libcuda link),
+// kernel launch with programmatic dependent launch enabled, and per-context
+// state that several host threads may set up at once.
 #pragma once
 
 #include <cuda.h>
@@ -8,19 +9,21 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 namespace nvfp4 {
 namespace tc {
 
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // (a function-local static is initialised once, also under concurrent first calls)
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult qr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
         qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+  }();
   return fn;
 }
 
@@ -71,6 +74,72 @@ inline cudaError_t launch_pdl(const void* func, dim3 grid, dim3 block, size_t sm
   cfg.numAttrs = 1;
   return cudaLaunchKernelExC(&cfg, func, args);
 }
+
+// Unique id of the CUDA context current on this host thread, 0 when none is
+// current yet (cuCtxGetCurrent / cuCtxGetId through the driver entry points).
+// Ids are never reused, so state keyed by them cannot outlive its context
+// (cudaDeviceReset, or a caller that makes another context current).
+inline cudaError_t current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (!get_current || !get_id) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  *id = 0;
+  if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  return cudaSuccess;
+}
+
+// The largest dynamic shared memory a kernel has been allowed
+// (cudaFuncAttributeMaxDynamicSharedMemorySize) in each context it ran in.
+// The attribute belongs to the kernel's module in one context, so it is
+// recorded per context id; the limit only ever grows, under a lock, so a
+// launch that needs less never lowers the limit another thread set for a
+// larger one.
+class SmemOptIn {
+ public:
+  cudaError_t ensure(const void* func, int bytes) {
+    unsigned long long ctx = 0;
+    cudaError_t e = current_context_id(&ctx);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu_);
+    for (int i = 0; i < used_; ++i)
+      if (ctx != 0 && slot_[i].ctx == ctx && slot_[i].bytes >= bytes) return cudaSuccess;
+    // (this also creates the device's primary context when none was current)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (ctx == 0 && (e = current_context_id(&ctx)) != cudaSuccess) return e;
+    for (int i = 0; i < used_; ++i)
+      if (slot_[i].ctx == ctx) {
+        slot_[i].bytes = bytes > slot_[i].bytes ? bytes : slot_[i].bytes;
+        return cudaSuccess;
+      }
+    slot_[used_ < kSlots ? used_++ : (next_++ % kSlots)] = {ctx, bytes};
+    return cudaSuccess;
+  }
+
+ private:
+  static constexpr int kSlots = 64;
+  struct Slot {
+    unsigned long long ctx;
+    int bytes;
+  };
+  std::mutex mu_;
+  Slot slot_[kSlots] = {};
+  int used_ = 0, next_ = 0;
+};
 
 }  // namespace tc
 }  // namespace nvfp4

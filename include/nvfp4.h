@@ -195,8 +195,12 @@ NVFP4_API size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *   NVFP4_GEMM_NOALLOC_SCRATCH_BYTES are rejected with NVFP4_ERR_WORKSPACE
  *   and launch nothing; every shape with M <= 1024 and M * K <= 2^22 fits
  *   (e.g. M = 512, K = 8192).
- * Set-up: the first call on each device (with that device current) looks up
- *   the array's device address; make it before any stream capture begins.
+ * Set-up: the first call in each CUDA context (normally the device's primary
+ *   context, current when the call is made) looks up the array's device
+ *   address and caches it under the context's unique id; make that call
+ *   before any stream capture in the context begins.  A call in a new context
+ *   (after cudaDeviceReset, or with another context made current) looks the
+ *   address up again.
  * Sharing: every call on a device uses the same array, which keeps what the
  *   last call wrote (nothing in it needs to start at zero).  Calls whose work
  *   overlaps on the GPU race on it: order them (e.g. one stream).
