@@ -3,9 +3,11 @@
 One step = one pass of every kernel of the hot path over the 27B-class layer
 (hidden 5120, MLP 17408), inputs resident in HBM:
   * quantize: nvfp4_amax + nvfp4_quantize of a BF16 [17408, 5120] N(0, 0.02) tensor
+  * quantize_mse: the same with the micro-scale search (nvfp4_quantize_mse)
   * gemv:     batch-1 decode GEMV, NVFP4 W [17408, 5120] (headline: HBM GB/s)
   * gemm_m32: 32-user decode GEMM, X [32, 5120]
   * gemm_m512: 512-token prefill GEMM, X [512, 5120]
+  * gemv_down: the MLP down projection W [5120, 17408], split-K decode GEMV
 Each kernel row is a CUDA graph of several launches over rotating weight copies
 (more bytes than the 126 MB L2 between two reads of one copy), timed with CUDA
 events on the launching stream.  `value` is the decode GEMV's algorithmic HBM
@@ -67,6 +69,9 @@ def w4a4_gemm_bytes(M: int, N: int, K: int) -> int:
     return N * K // 2 + N * K // 16 + M * K // 2 + M * K // 16 + 2 * M * N + 8
 
 
+MSE_WINDOW = 8                  # E4M3 codes either side of the round-to-nearest scale
+MSE_FP64_OPS_PER_CANDIDATE = 64  # 16 elements x (multiply, subtract, square, add)
+
 FP4_PER_BF16 = 4  # nominal dense FP4 / BF16 tensor throughput of B200 (9 / 2.25 PFLOP/s)
 
 MOE = {"E": 128, "N": 1536, "K": 2048, "top": 8}  # synthetic MoE layer: stacked experts, top-8 routing, one token
@@ -102,12 +107,14 @@ _CSRC = "gemm_decode_nvfp4_b200/csrc/"
 KERNEL_SOURCES = {
     "gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh"],
+    "quantize_mse": [_CSRC + "quantize.cu", _CSRC + "nvfp4_device.cuh"],
     "gemm_m32": [_CSRC + "gemm_small.cu", _CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh",
                  _CSRC + "tc_host.h"],
     "gemm_m512": [_CSRC + "gemm_tc.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh"],
     "mx_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh"],
     "moe_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "gemv_down": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "w4a4_m512": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
                   _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "w4a4_gemm": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
@@ -128,6 +135,16 @@ def traffic_from_profiles(row: str):
     if not e or e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[row]):
         return None
     return e.get("dram_bytes_per_call")
+
+
+def dram_attested(traffic_bytes, us: float, hbm_gbs: float) -> dict:
+    """GB/s and fraction of the HBM peak that a row's measured DRAM bytes per
+    call (read + write, from ncu) give over its CUDA-event time; None without a
+    current traffic figure."""
+    if not traffic_bytes:
+        return {"GB/s_dram": None, "frac_hbm_dram": None}
+    gbs = traffic_bytes / (us * 1e-6) / 1e9
+    return {"GB/s_dram": gbs, "frac_hbm_dram": gbs / hbm_gbs}
 
 
 # ------------------------------------------------------------ ranks (replicas)
@@ -306,10 +323,28 @@ def run_gpu(args):
         for i in range(copies):
             nv.gemv_grouped(moe_x, moe_q, moe_s, moe_g, moe_ids[i], moe_tok, moe_y)
 
+    # MLP down projection of the same layer, W [5120, 17408]: few rows, long K,
+    # the split-K decode GEMV (the library's choice of split), 8 copies (400 MB)
+    dcfg = workloads.CONFIGS["down"]
+    dq0, ds0, dg0 = nv.quantize_new(workloads.weight_bf16(dcfg).to(dev))
+    dqs = [dq0] + [dq0.clone() for _ in range(copies - 1)]
+    dss = [ds0] + [ds0.clone() for _ in range(copies - 1)]
+    xdown = workloads.activations(1, dcfg.K, dcfg.seed).to(dev).reshape(-1)
+    ydown = [torch.empty((dcfg.N,), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+
+    def gemv_down_all():
+        for i in range(copies):
+            nv.gemv(xdown, dqs[i], dss[i], dg0, ydown[i], static_weights=True)
+
     def quant_all():
         amax_buf.zero_()
         nv.amax(wq_in, amax_buf)
         nv.quantize(wq_in, qq, sq, gq, amax=amax_buf)
+
+    def quant_mse_all():  # the same tensor, micro-scale search over +-8 E4M3 codes
+        amax_buf.zero_()
+        nv.amax(wq_in, amax_buf)
+        nv.quantize_mse(wq_in, qq, sq, gq, amax=amax_buf, window=8)
 
     # W4A4 prefill (NVFP4 activations): the same 8 weight copies, scales
     # rearranged once for the block-scaled tensor cores
@@ -330,6 +365,7 @@ def run_gpu(args):
                 nv.w4a4_gemm(w4_qx, w4_sx, w4_amax, qs[i], smmas[i], g0, Y512w, static_weights=True)
 
     rows.append(("quantize", quant_all, 1, 2))
+    rows.append(("quantize_mse", quant_mse_all, 1, 2))
     rows.append(("mx_quantize", mx_quant_all, 1, 1))
     if gemm_ok:
         def m32_all():
@@ -348,6 +384,7 @@ def run_gpu(args):
         rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
     rows.append(("mx_gemv", mx_gemv_all, copies, 1))
     rows.append(("moe_gemv", moe_all, copies, 1))
+    rows.append(("gemv_down", gemv_down_all, copies, 1))
     rows.append(("gemv_ordered", gemv_ordered_all, copies, 1))
     rows.append(("gemv", gemv_all, copies, 1))
     if args.only != "all":  # profiling runs: keep only the named row (plus the headline GEMV)
@@ -376,7 +413,7 @@ def run_gpu(args):
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = torch.ones((2 * l2_bytes // 4,), dtype=torch.float32, device=dev)
     flush_out = torch.empty((), dtype=torch.float32, device=dev)
-    flush_after = ("quantize", "mx_quantize")
+    flush_after = ("quantize", "quantize_mse", "mx_quantize")
 
     def l2_writeback():
         torch.sum(flush_buf, dim=0, out=flush_out)
@@ -412,9 +449,12 @@ def run_gpu(args):
 
     total_ms = step_start.elapsed_time(step_end)
     per_launch_ms = {}
+    spread = {}
     for name, _, launches, _ in rows:
-        t = sum(a.elapsed_time(b) for a, b in evs[name])
-        per_launch_ms[name] = t / (args.steps * launches)
+        per_step = [a.elapsed_time(b) / launches for a, b in evs[name]]
+        per_launch_ms[name] = sum(per_step) / args.steps
+        q = statistics.quantiles(per_step, n=10) if len(per_step) >= 2 else [per_step[0]] * 9
+        spread[name] = {"p10_us": q[0] * 1e3, "median_us": statistics.median(per_step) * 1e3, "p90_us": q[-1] * 1e3}
 
     red = max_over_ranks([total_ms] + [per_launch_ms[n] for n, *_ in rows], world, dev)
     total_ms = red[0]
@@ -450,6 +490,22 @@ def run_gpu(args):
         kernels["moe_gemv"] = {"us": per_launch_ms["moe_gemv"] * 1e3, "GB/s": mg, "frac_hbm": mg / hbm, "bytes": mb,
                                "workload": f"grouped decode GEMV: {MOE['top']} of {MOE['E']} stacked experts "
                                            f"[{MOE['N']}, {MOE['K']}], one token, synthetic routing"}
+    if "quantize_mse" in per_launch_ms:
+        qb = quantize_bytes(N, K)
+        t_mse = per_launch_ms["quantize_mse"] * 1e3
+        kernels["quantize_mse"] = {
+            "us": t_mse, "GB/s": qb / (t_mse * 1e-6) / 1e9, "bytes": qb,
+            "x_round_to_nearest": t_mse / kernels["quantize"]["us"] if "quantize" in kernels else None,
+            "fp64_ops_per_block_max": MSE_FP64_OPS_PER_CANDIDATE * (2 * MSE_WINDOW + 1),
+            "what": "amax + micro-scale search quantizer (E4M3 candidates within 8 codes, fp64 error): "
+                    "FP64-bound; the pages report about 6x the round-to-nearest cost"}
+    if "gemv_down" in per_launch_ms:
+        db = gemv_bytes(dcfg.N, dcfg.K)
+        dgbs = db / (per_launch_ms["gemv_down"] * 1e-3) / 1e9
+        kernels["gemv_down"] = {"us": per_launch_ms["gemv_down"] * 1e3, "GB/s": dgbs, "frac_hbm": dgbs / hbm,
+                                "bytes": db, "weight_bytes_per_token": dcfg.N * dcfg.K // 2 + dcfg.N * dcfg.K // 16,
+                                "workload": f"down-projection decode GEMV W [{dcfg.N}, {dcfg.K}] x BF16 [1, {dcfg.K}]",
+                                "launch": "split-K (library's choice), static weights, 8 copies per graph"}
     if "mx_quantize" in per_launch_ms:
         mb = mx_quantize_bytes(N, K)
         mq = mb / (per_launch_ms["mx_quantize"] * 1e-3) / 1e9
@@ -507,6 +563,14 @@ def run_gpu(args):
     for name in kernels:
         if "us" in kernels[name]:
             kernels[name]["traffic"] = traffic_from_profiles(name)
+            if name in spread:
+                kernels[name]["spread"] = spread[name]
+    for name in ("quantize", "mx_quantize"):
+        # the quantizers' output is still in L2 when their events end: beside the
+        # algorithmic fraction, the fraction that the DRAM bytes ncu measured for
+        # the same row support
+        if name in kernels:
+            kernels[name].update(dram_attested(kernels[name]["traffic"], kernels[name]["us"], hbm))
     traffic = kernels["gemv"]["traffic"]
     out = None
     if rank == 0:
@@ -526,9 +590,9 @@ def run_gpu(args):
             "config": {"workload": WORKLOAD, "N": N, "K": K, "M": 1, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {copies} rotating weight copies "
                              f"({copies * (N * K // 2 + N * K // 16) / 1e6:.0f} MB) per graph",
-                       "row_order": "quantize, MXFP4 quantize (each followed by an untimed read of 2 x L2 that writes back their dirty output), gemm M=512, W4A4 M=512 (step), W4A4 GEMM, gemm M=32, MXFP4 gemv, MoE gemv, gemv ordered, gemv static: each GEMV graph "
+                       "row_order": "quantize, MSE quantize, MXFP4 quantize (each followed by an untimed read of 2 x L2 that writes back their dirty output), gemm M=512, W4A4 M=512 (step), W4A4 GEMM, gemm M=32, MXFP4 gemv, MoE gemv, down-projection gemv, gemv ordered, gemv static: each GEMV graph "
                                     "follows GEMVs, not the rows that leave tens of MB of dirty output in L2",
-                       "step": "quantize [17408,5120] (NVFP4, MXFP4) + gemm M=512 + W4A4 M=512 (quantize X + GEMM) + W4A4 GEMM + gemm M=32 + MXFP4 gemv + grouped MoE gemv + gemv M=1 (x2: ordered and static-weights)",
+                       "step": "quantize [17408,5120] (NVFP4 round-to-nearest, NVFP4 micro-scale search, MXFP4) + gemm M=512 + W4A4 M=512 (quantize X + GEMM) + W4A4 GEMM + gemm M=32 + MXFP4 gemv + grouped MoE gemv + down-projection gemv [5120, 17408] (split-K) + gemv M=1 (x2: ordered and static-weights)",
             "gemv_launch": "8 GEMVs per graph on 8 weight copies, programmatic dependent launch (static weights)"},
             "roofline": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemv_gbs / hbm, "traffic": traffic,
@@ -616,15 +680,15 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--copies", type=int, default=8, help="rotating weight copies per graph (L2 defeat)")
     ap.add_argument("--cpu-rows", type=int, default=17408)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "gemm_m32",
+    ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "quantize_mse", "gemm_m32",
                                                       "gemm_m512", "mx_gemv", "mx_quantize", "moe_gemv",
-                                                      "w4a4_m512", "w4a4_gemm"],
+                                                      "gemv_down", "w4a4_m512", "w4a4_gemm"],
                     help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps

@@ -19,7 +19,7 @@ import re
 import torch
 
 __all__ = [
-    "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "gemv", "gemm",
+    "Nvfp4Error", "LIB_PATH", "lib", "version", "amax", "quantize", "quantize_mse", "gemv", "gemm",
     "gemm_workspace_size", "quantize_new", "linear", "declared_symbols", "check_device_errors",
     "FLAG_STATIC_WEIGHTS", "gemm_noalloc", "GEMM_NOALLOC_SCRATCH_BYTES",
     "mx_quantize", "mx_quantize_new", "mx_gemv", "gemv_grouped", "mx_to_nvfp4",
@@ -44,6 +44,7 @@ lib.nvfp4_last_error.argtypes, lib.nvfp4_last_error.restype = [], ctypes.c_char_
 lib.nvfp4_status_string.argtypes, lib.nvfp4_status_string.restype = [ctypes.c_int], ctypes.c_char_p
 lib.nvfp4_amax.argtypes = [_p, _i64, _i64, _i64, _p, _p]
 lib.nvfp4_quantize.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _p]
+lib.nvfp4_quantize_mse.argtypes = [_p, _i64, _i64, _i64, _p, ctypes.c_int32, _p, _p, _p, _p]
 lib.nvfp4_gemv.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, _p]
 lib.nvfp4_gemm.argtypes = [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]
 lib.nvfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
@@ -65,7 +66,7 @@ lib.mxfp4_gemv.argtypes = [_p, _p, _p, _p, _i64, _i64, _p]
 lib.mxfp4_gemv_ex.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_uint32, _p]
 lib.nvfp4_gemm_workspace_size.restype = _sz
 lib.nvfp4_check_device_errors.argtypes = []
-for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
+for _f in (lib.nvfp4_amax, lib.nvfp4_quantize, lib.nvfp4_quantize_mse, lib.nvfp4_gemv, lib.nvfp4_gemm, lib.nvfp4_gemv_ex, lib.nvfp4_gemm_ex,
            lib.nvfp4_gemm_noalloc, lib.nvfp4_check_device_errors, lib.mxfp4_quantize, lib.mxfp4_gemv,
            lib.mxfp4_gemv_ex, lib.nvfp4_gemv_grouped, lib.mxfp4_to_nvfp4_scales,
            lib.nvfp4_w4a4_prepare_weights, lib.nvfp4_w4a4_quantize_x, lib.nvfp4_w4a4_gemm,
@@ -175,13 +176,41 @@ def quantize(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch.Ten
           _stream(stream, dev))
 
 
+def quantize_mse(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch.Tensor | None,
+                 amax: torch.Tensor | None = None, window: int = 8, stream=None) -> None:
+    """NVFP4 of BF16 w [N, K] with each micro-scale chosen by the least fp64
+    reconstruction error among the E4M3 codes within `window` of the
+    round-to-nearest one (nvfp4_quantize_mse); otherwise as quantize()."""
+    _need(w, torch.bfloat16, "w", 2)
+    _need(q, torch.uint8, "q", 2)
+    _need(s, torch.uint8, "s", 2)
+    N, K = w.shape
+    if q.shape != (N, K // 2) or s.shape != (N, K // 16) or not q.is_contiguous() or not s.is_contiguous():
+        raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
+    if g_out is not None:
+        _need(g_out, torch.float32, "g_out")
+    if amax is not None:
+        _need(amax, torch.float32, "amax")
+    dev = _device(w, q, s, g_out, amax)
+    _call("nvfp4_quantize_mse", dev, _ptr(w), N, K, w.stride(0), _ptr(amax), int(window), _ptr(q), _ptr(s),
+          _ptr(g_out), _stream(stream, dev))
+
+
 FLAG_STATIC_WEIGHTS = 1
 
 
+def _ksplit_flag(k_split: int) -> int:
+    """NVFP4_FLAG_KSPLIT(k_split): 0 = the library's choice, else 1, 2, 4 or 8."""
+    if k_split not in (0, 1, 2, 4, 8):
+        raise ValueError(f"k_split must be 0, 1, 2, 4 or 8, got {k_split}")
+    return k_split << 8
+
+
 def gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, y: torch.Tensor,
-         stream=None, static_weights: bool = False) -> None:
+         stream=None, static_weights: bool = False, k_split: int = 0) -> None:
     """y[N] = bf16(g * W_deq . x) for BF16 x [K] (or [1, K]).  static_weights: q, s, g
-    are not written by work still running on the stream (see NVFP4_FLAG_STATIC_WEIGHTS)."""
+    are not written by work still running on the stream (see NVFP4_FLAG_STATIC_WEIGHTS).
+    k_split: CTAs of a cluster that split K (NVFP4_FLAG_KSPLIT); 0 = chosen per shape."""
     _need(x, torch.bfloat16, "x")
     _need(q, torch.uint8, "q", 2)
     _need(s, torch.uint8, "s", 2)
@@ -192,7 +221,7 @@ def gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: torch.Tensor, y: 
         raise ValueError("x must hold K and y N contiguous elements")
     if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 16):
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/16]")
-    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    flags = (FLAG_STATIC_WEIGHTS if static_weights else 0) | _ksplit_flag(k_split)
     dev = _device(x, q, s, g, y)
     _call("nvfp4_gemv_ex", dev, _ptr(x), _ptr(q), _ptr(s), _ptr(g), _ptr(y), N, K, flags, _stream(stream, dev))
 
@@ -309,8 +338,8 @@ def mx_quantize_new(w: torch.Tensor, stream=None):
 
 
 def mx_gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, y: torch.Tensor, stream=None,
-            static_weights: bool = False) -> None:
-    """y[N] = bf16(W_deq . x) for MXFP4 weights and BF16 x [K]."""
+            static_weights: bool = False, k_split: int = 0) -> None:
+    """y[N] = bf16(W_deq . x) for MXFP4 weights and BF16 x [K]; k_split as for gemv()."""
     _need(x, torch.bfloat16, "x")
     _need(q, torch.uint8, "q", 2)
     _need(s, torch.uint8, "s", 2)
@@ -320,7 +349,7 @@ def mx_gemv(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, y: torch.Tensor, 
         raise ValueError("x must hold K and y N contiguous elements")
     if not q.is_contiguous() or not s.is_contiguous() or s.shape != (N, K // 32):
         raise ValueError("q/s must be contiguous [N, K/2] / [N, K/32]")
-    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    flags = (FLAG_STATIC_WEIGHTS if static_weights else 0) | _ksplit_flag(k_split)
     dev = _device(x, q, s, y)
     _call("mxfp4_gemv_ex", dev, _ptr(x), _ptr(q), _ptr(s), _ptr(y), N, K, flags, _stream(stream, dev))
 

@@ -36,6 +36,14 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 constexpr uint32_t kKnownFlags = NVFP4_FLAG_STATIC_WEIGHTS;
+constexpr uint32_t kGemvFlags = NVFP4_FLAG_STATIC_WEIGHTS | NVFP4_FLAG_KSPLIT_MASK;
+
+// The K split a decode GEMV call asks for (0 = the library's choice), or -1
+// for a value other than 1, 2, 4, 8.
+int ksplit_of(uint32_t flags) {
+  const int c = (int)((flags & NVFP4_FLAG_KSPLIT_MASK) >> 8);
+  return (c == 0 || c == 1 || c == 2 || c == 4 || c == 8) ? c : -1;
+}
 
 constexpr int kMaxDevices = 64;
 int g_dev_state[kMaxDevices];  // 0 unknown, 1 ok, 2 unsupported
@@ -117,9 +125,14 @@ nvfp4_status nvfp4_amax(const uint16_t* w, int64_t rows, int64_t cols, int64_t l
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "amax launch");
 }
 
-nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
-                            const float* amax, uint8_t* q, uint8_t* s, float* g_out,
-                            nvfp4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// nvfp4_quantize (window < 0) and nvfp4_quantize_mse (window >= 0): same
+// arguments, same checks, the same amax handling.
+nvfp4_status quantize_any(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, const float* amax, uint8_t* q,
+                          uint8_t* s, float* g_out, nvfp4_stream_t stream, int window) {
   nvfp4_status st = check_k(K);
   if (st != NVFP4_OK) return st;
   if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
@@ -143,17 +156,37 @@ nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw
   if (st != NVFP4_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e;
+  auto quant = [&](const float* a, float* gout) {
+    return window < 0 ? nvfp4::launch_quantize(w, N, K, ldw, a, q, s, gout, cs, sms)
+                      : nvfp4::launch_quantize_mse(w, N, K, ldw, a, window, q, s, gout, cs, sms);
+  };
   if (amax) {
-    e = nvfp4::launch_quantize(w, N, K, ldw, amax, q, s, g_out, cs, sms);
+    e = quant(amax, g_out);
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "quantize launch");
   }
   // g_out first accumulates this tensor's amax, then is overwritten with g.
   if ((e = cudaMemsetAsync(g_out, 0, sizeof(float), cs)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   if (N > 0 && (e = nvfp4::launch_amax(w, N, K, ldw, g_out, cs, sms)) != cudaSuccess) return cuda_fail(e, "amax launch");
-  if ((e = nvfp4::launch_quantize(w, N, K, ldw, g_out, q, s, nullptr, cs, sms)) != cudaSuccess)
-    return cuda_fail(e, "quantize launch");
+  if ((e = quant(g_out, nullptr)) != cudaSuccess) return cuda_fail(e, "quantize launch");
   if ((e = nvfp4::launch_finalize_scale(g_out, cs)) != cudaSuccess) return cuda_fail(e, "finalize launch");
   return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                            const float* amax, uint8_t* q, uint8_t* s, float* g_out,
+                            nvfp4_stream_t stream) {
+  return quantize_any(w, N, K, ldw, amax, q, s, g_out, stream, -1);
+}
+
+nvfp4_status nvfp4_quantize_mse(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, const float* amax,
+                                int32_t window, uint8_t* q, uint8_t* s, float* g_out, nvfp4_stream_t stream) {
+  if (window < 0 || window > 125)
+    return fail(NVFP4_ERR_INVALID_ARG, "window=%d must be in 0..125 (E4M3 codes either side)", (int)window);
+  return quantize_any(w, N, K, ldw, amax, q, s, g_out, stream, window);
 }
 
 nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
@@ -163,7 +196,9 @@ nvfp4_status nvfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
 
 nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
                            uint16_t* y, int64_t N, int64_t K, uint32_t flags, nvfp4_stream_t stream) {
-  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~kGemvFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int splits = ksplit_of(flags);
+  if (splits < 0) return fail(NVFP4_ERR_INVALID_ARG, "NVFP4_FLAG_KSPLIT(c) needs c in {1, 2, 4, 8}");
   nvfp4_status st = check_k(K);
   if (st != NVFP4_OK) return st;
   if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
@@ -183,8 +218,12 @@ nvfp4_status nvfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
   const bool static_w = (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0;
+  if (splits > 1 && !nvfp4::gemv_split_fits(N, K, sms, false, splits))
+    return fail(NVFP4_ERR_SHAPE, "a K split of %d does not fit N=%lld K=%lld (it needs K %% 256 == 0, at least %d "
+                "512-element columns, and at most 11520 elements of x per CTA)", splits, (long long)N, (long long)K,
+                splits);
   cudaError_t e;
-  e = nvfp4::launch_gemv(x, q, s, g, y, N, K, sms, static_w, (cudaStream_t)stream);
+  e = nvfp4::launch_gemv(x, q, s, g, y, N, K, sms, static_w, (cudaStream_t)stream, splits);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "gemv launch");
 }
 
@@ -267,7 +306,9 @@ nvfp4_status mxfp4_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, u
 
 nvfp4_status mxfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
                            int64_t K, uint32_t flags, nvfp4_stream_t stream) {
-  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~kGemvFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const int splits = ksplit_of(flags);
+  if (splits < 0) return fail(NVFP4_ERR_INVALID_ARG, "NVFP4_FLAG_KSPLIT(c) needs c in {1, 2, 4, 8}");
   if (K <= 0 || K % 32 != 0) return fail(NVFP4_ERR_SHAPE, "K=%lld must be a positive multiple of 32", (long long)K);
   if (N < 0) return fail(NVFP4_ERR_SHAPE, "N=%lld < 0", (long long)N);
   if (K > nvfp4::kGemvMaxK) return fail(NVFP4_ERR_SHAPE, "K=%lld exceeds the GEMV limit %lld", (long long)K, (long long)nvfp4::kGemvMaxK);
@@ -285,7 +326,11 @@ nvfp4_status mxfp4_gemv_ex(const uint16_t* x, const uint8_t* q, const uint8_t* s
   nvfp4_status st = check_device(&sms);
   if (st != NVFP4_OK) return st;
   const bool static_w = (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0;
-  cudaError_t e = nvfp4::launch_gemv_mx(x, q, s, y, N, K, sms, static_w, (cudaStream_t)stream);
+  if (splits > 1 && !nvfp4::gemv_split_fits(N, K, sms, true, splits))
+    return fail(NVFP4_ERR_SHAPE, "a K split of %d does not fit N=%lld K=%lld (it needs K %% 512 == 0, at least %d "
+                "512-element columns, and at most 11520 elements of x per CTA)", splits, (long long)N, (long long)K,
+                splits);
+  cudaError_t e = nvfp4::launch_gemv_mx(x, q, s, y, N, K, sms, static_w, (cudaStream_t)stream, splits);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "mxfp4 gemv launch");
 }
 

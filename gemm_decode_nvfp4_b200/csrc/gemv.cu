@@ -421,11 +421,11 @@ constexpr int kRingConsumers = kRingConsumerWarps * 32;   // 480 threads
 constexpr int kRingThreads = kRingConsumers + 32;         // 512 threads x 64 registers: half an SM
 constexpr int kRingBK = 256;                              // code bytes of a row per stage (512 weights)
 constexpr int kRingChunks = kRingBK / 16;                 // 16 lanes share a row
-constexpr int kRingRows = 4;                              // rows per lane
-constexpr int kRingMaxBR = (kRingConsumers / kRingChunks) * kRingRows;  // 120 rows per stage
-constexpr int kRingScOff = kRingMaxBR * kRingBK;          // scales start after a fixed 120-row code block
-constexpr int kRingStage = kRingScOff + kRingMaxBR * (kRingBK / 8);   // 34560 bytes
-constexpr int kRingMaxK = kRingConsumers * 24;            // x: at most 3 uint4 per consumer thread
+constexpr int kRingSlots = kRingConsumers / kRingChunks;  // 30 row slots: a lane owns rows slot + 30 i
+constexpr int kRingRows = 4;                              // rows per lane at most
+constexpr int kRingMaxBR = kRingSlots * kRingRows;        // 120 rows per stage
+constexpr int kRingMaxSlice = kRingConsumers * 24;        // x elements per CTA: at most 3 uint4 per consumer
+constexpr int kRingMaxStages = 8;
 constexpr uint64_t kRingWaitNs = 2000000000ull;
 
 __device__ __forceinline__ void ring_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
@@ -439,32 +439,73 @@ __device__ __forceinline__ void tma_load_3d_evict_first(void* dst, const void* t
       : "memory");
 }
 
-// Shared memory: S stages of kRingStage bytes, then x (nks x 1 KB: f16, each
-// stage's 512 values laid out [word i][chunk c] so that a quarter-warp reads
-// 128 contiguous bytes), then the barriers and the reduction scratch.
-// Rows of a CTA: [blockIdx.x * nblk * BR, + nblk * BR), in nblk blocks of BR
-// rows (BR <= 120) that go through the ring one 256-byte column at a time.
+// Exact fp32 dot product of weight row `row` with x over k in [k0, k1) (block
+// boundaries), one warp, x read as BF16 from global memory: the path for x
+// outside the f16 window.  Every lane returns the sum.
+template <bool MX>
+__device__ __noinline__ float dot_exact_range(const uint16_t* __restrict__ x, const uint8_t* __restrict__ q,
+                                              const uint8_t* __restrict__ s, int K, int row, int k0, int k1) {
+  constexpr int BS = MX ? 32 : 16;  // elements per scale
+  const int lane = threadIdx.x & 31;
+  const uint8_t* qr = q + (int64_t)row * (K / 2);
+  const uint8_t* sr = s + (int64_t)row * (K / BS);
+  float acc = 0.0f;
+  for (int b = k0 / BS + lane; b < k1 / BS; b += 32) {
+    float2 p = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int i = 0; i < BS / 8; ++i) {  // 8 weights (4 code bytes) at a time
+      const uint32_t wd = *reinterpret_cast<const uint32_t*>(qr + (BS / 2) * b + 4 * i);
+      const uint4 xa = *reinterpret_cast<const uint4*>(x + BS * b + 8 * i);
+      p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<0>(wd)), make_float2(bf16lo_to_float(xa.x), bf16hi_to_float(xa.x)), p);
+      p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<1>(wd)), make_float2(bf16lo_to_float(xa.y), bf16hi_to_float(xa.y)), p);
+      p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<2>(wd)), make_float2(bf16lo_to_float(xa.z), bf16hi_to_float(xa.z)), p);
+      p = __ffma2_rn(f16x2_to_float2(e2m1x2_byte_to_f16x2<3>(wd)), make_float2(bf16lo_to_float(xa.w), bf16hi_to_float(xa.w)), p);
+    }
+    acc = fmaf(p.x + p.y, MX ? e8m0_to_float(sr[b]) : e4m3_to_float(sr[b]), acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  return acc;
+}
+
+// Shared memory: S stages of SB bytes (a stage: BR rows x 256 code bytes, then
+// their BR x 32 (NVFP4) or 16 (MXFP4) scale bytes), then x (ncx x 1 KB: f16,
+// each stage column's 512 values laid out [word i][chunk c] so that a
+// quarter-warp reads 128 contiguous bytes), then the barriers, the reduction
+// scratch and (K split over a cluster) the fp32 partial of each row.
+// Rows of a CTA: [cl * nblk * BR, + nblk * BR) for cluster cl = blockIdx.x / C,
+// in nblk blocks of BR rows (BR <= 120) that go through the ring one 256-byte
+// column at a time.  K: the nks = ceil(K / 512) columns are split over the C
+// CTAs of a cluster (rank r takes columns [r nks / C, (r + 1) nks / C)); with
+// C > 1 each CTA leaves its rows' partial sums in shared memory and the
+// cluster adds them in rank order (fixed order: deterministic).
 template <bool MX, bool GROUPED>
 __global__ void __launch_bounds__(kRingThreads, 2)
     gemv_ring_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
                      const uint16_t* __restrict__ x, const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
                      const float* __restrict__ g, uint16_t* __restrict__ y, int N, int K, int BR, int nblk,
-                     int S, Problems P) {
+                     int S, int SB, int C, Problems P) {
   extern __shared__ __align__(1024) uint8_t sm[];
   constexpr int kSB = MX ? kRingBK / 16 : kRingBK / 8;  // scale bytes of a row per stage
-  const int nks = (K / 2 + kRingBK - 1) / kRingBK;  // stages per row block
+  const int nks = (K / 2 + kRingBK - 1) / kRingBK;      // stage columns of a row
+  const int ncx = (nks + C - 1) / C;                    // most columns a CTA takes
+  const int rank = C > 1 ? (int)ptx::cluster_ctarank() : 0;
+  const int t0 = (int)((int64_t)rank * nks / C), t1 = (int)((int64_t)(rank + 1) * nks / C);
+  const int ncols = t1 - t0;
+  const int k0 = t0 * 2 * kRingBK, k1 = min(t1 * 2 * kRingBK, K);  // this CTA's x elements
   uint8_t* ring = sm;
-  uint4* xs = reinterpret_cast<uint4*>(sm + S * kRingStage);
-  uint64_t* full = reinterpret_cast<uint64_t*>(xs + nks * 64);
+  uint4* xs = reinterpret_cast<uint4*>(sm + S * SB);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xs + ncx * 64);
   uint64_t* empty = full + S;
   uint64_t* xfull = empty + S;
-  uint32_t* red = reinterpret_cast<uint32_t*>(xfull + 1);        // [2][16]
+  uint32_t* red = reinterpret_cast<uint32_t*>(xfull + 1);        // [2][16], then two flags
   volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 32);
+  float* part = reinterpret_cast<float*>(red + 36);               // [nblk * BR], used when C > 1
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int row_base = blockIdx.x * nblk * BR;
+  const int row_base = (blockIdx.x / C) * nblk * BR;
   const int nb_here = min(nblk, (N - row_base + BR - 1) / BR);
-  const int total = nb_here * nks;
+  const int total = nb_here * ncols;
 
   if (tid == 0) {
     for (int i = 0; i < S; ++i) {
@@ -473,6 +514,7 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     }
     ptx::mbar_init(xfull, 1);
     *abort_flag = 0;
+    red[33] = 0;
     ptx::fence_mbar_init();
   }
   __syncthreads();
@@ -486,25 +528,25 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     int n = 0, slot = 0, t = 0, rb = 0, e_id = 0;
     uint32_t phase = 0;
     auto issue = [&]() {
-      uint8_t* dst = ring + slot * kRingStage;
+      uint8_t* dst = ring + slot * SB;
       const int row0 = row_base + rb * BR;
       ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)BR * (kRingBK + kSB));
-      tma_load_3d_evict_first(dst, &tq, &full[slot], t * kRingBK, row0, e_id, policy);
-      tma_load_3d_evict_first(dst + kRingScOff, &ts, &full[slot], t * kSB, row0, e_id, policy);
+      tma_load_3d_evict_first(dst, &tq, &full[slot], (t0 + t) * kRingBK, row0, e_id, policy);
+      tma_load_3d_evict_first(dst + BR * kRingBK, &ts, &full[slot], (t0 + t) * kSB, row0, e_id, policy);
       if (++slot == S) { slot = 0; phase ^= 1; }
-      if (++t == nks) { t = 0; ++rb; }
+      if (++t == ncols) { t = 0; ++rb; }
     };
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x, ids and the weights only after this
     int tok = 0;
     if (!resolve_problem<GROUPED>(P, e_id, tok)) return;  // nothing issued: the consumers write zeros
-    ptx::mbar_arrive_expect_tx(xfull, (uint32_t)K * 2);
-    ptx::bulk_load(xs, x + (int64_t)tok * P.x_stride, (uint32_t)K * 2, xfull);
+    ptx::mbar_arrive_expect_tx(xfull, (uint32_t)(k1 - k0) * 2);
+    ptx::bulk_load(xs, x + (int64_t)tok * P.x_stride + k0, (uint32_t)(k1 - k0) * 2, xfull);
     for (; n < total; ++n) {
       if (n >= S) {  // wait until the consumers have released this slot (or have given up on the ring)
         bool ok = ptx::mbar_try_wait(&empty[slot], phase ^ 1);
-        const uint64_t t0 = ok ? 0 : ptx::globaltimer_ns();
+        const uint64_t tw = ok ? 0 : ptx::globaltimer_ns();
         while (!ok && !*abort_flag) {
-          if (ptx::globaltimer_ns() - t0 > kRingWaitNs) {
+          if (ptx::globaltimer_ns() - tw > kRingWaitNs) {
             atomicAdd(&g_gemv_wait_timeouts, 1u);
             break;
           }
@@ -538,57 +580,79 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     x += (int64_t)tok * P.x_stride;
     y += (int64_t)blockIdx.y * P.y_stride;
   }
+  const float gv = MX ? 1.0f : *g;
+  // Row (block rb, local row rl) gets its value: stored (C == 1) or left as a
+  // partial for the cluster.
+  auto emit = [&](int rb, int rl, float v) {
+    const int row = row_base + rb * BR + rl;
+    if (C > 1) {
+      part[rb * BR + rl] = v;
+    } else if (row < N) {
+      const __nv_bfloat16 o = __float2bfloat16_rn(v);
+      y[row] = *reinterpret_cast<const uint16_t*>(&o);
+    }
+  };
+  // x: a warp whose bounded wait gave up marks the CTA failed; every consumer
+  // thread then learns it at the barrier below (no warp leaves before it, so
+  // the barrier always completes)
+  volatile int* x_failed = reinterpret_cast<volatile int*>(red + 33);
   if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(xfull, 0, kRingWaitNs))) {
-    if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+    if (lane == 0) {
+      atomicAdd(&g_gemv_wait_timeouts, 1u);
+      *x_failed = 1;
+    }
     *abort_flag = 1;
-    return;
   }
-  // range of |x| over the raw BF16 bit patterns, which stay in registers
-  const int nx = K >> 3;
+  bool failed;  // a bounded wait gave up: the partials are NaN, nothing else runs
+  int e = 0;
+  bool fast = true;
+  const int nx = (k1 - k0) >> 3;  // x vectors of this CTA
   uint4 raw[3];
-  uint32_t mx = 0, mn = 0xFFFFu;
+  {
+    // range of |x| over the raw BF16 bit patterns, which stay in registers
+    uint32_t mx = 0, mn = 0xFFFFu;
 #pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    const int u = tid + k * kRingConsumers;
-    raw[k] = u < nx ? xs[u] : make_uint4(0, 0, 0, 0);
-    const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+    for (int k = 0; k < 3; ++k) {
+      const int u = tid + k * kRingConsumers;
+      raw[k] = u < nx ? xs[u] : make_uint4(0, 0, 0, 0);
+      const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
-      mx = max(mx, max(lo, hi));
-      mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
+        mx = max(mx, max(lo, hi));
+        mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
+      }
+    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+    if (lane == 0) { red[warp] = mx; red[16 + warp] = mn; }
+    ring_sync(kRingConsumers);  // every raw value is in registers: the buffer may be overwritten
+    failed = *x_failed != 0;
+    mx = red[0]; mn = red[16];
+#pragma unroll
+    for (int w = 1; w < kRingConsumerWarps; ++w) { mx = max(mx, red[w]); mn = min(mn, red[16 + w]); }
+    if (mx >= 0x7F80u) {
+      fast = false;
+    } else if (mx != 0) {
+      const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
+      e = 15 - hi_exp;
+      fast = hi_exp - lo_exp <= 32;
     }
   }
-  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-  mn = __reduce_min_sync(0xFFFFFFFFu, mn);
-  if (lane == 0) { red[warp] = mx; red[16 + warp] = mn; }
-  ring_sync(kRingConsumers);  // every raw value is in registers: the buffer may be overwritten
-  mx = red[0]; mn = red[16];
-#pragma unroll
-  for (int w = 1; w < kRingConsumerWarps; ++w) { mx = max(mx, red[w]); mn = min(mn, red[16 + w]); }
-  bool fast = true;
-  int e = 0;
-  if (mx >= 0x7F80u) {
-    fast = false;
-  } else if (mx != 0) {
-    const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
-    e = 15 - hi_exp;
-    fast = hi_exp - lo_exp <= 32;
-  }
-  const float gv = MX ? 1.0f : *g;
-  if (!fast) {  // x outside the f16 window: the producer stops, every warp takes rows exactly
+  if (!failed && !fast) {  // x outside the f16 window: the producer stops, every warp takes rows exactly
     *abort_flag = 1;
-    const int nrows = min(N - row_base, nblk * BR);
-    for (int r = warp; r < nrows; r += kRingConsumerWarps) rows_exact<MX>(x, q, s, g, y, N, K, row_base + r, 1);
+    const int nrows = min(N - row_base, nb_here * BR);
+    for (int r = warp; r < nrows; r += kRingConsumerWarps) {
+      const float v = dot_exact_range<MX>(x, q, s, K, row_base + r, k0, k1) * gv;
+      if (lane == 0) emit(r / BR, r % BR, v);
+    }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    return;
-  }
-  {
+  } else if (!failed) {
     const int e1 = e / 2, e2 = e - e1;  // two exact power-of-two steps
     const float m1 = exp2i(e1), m2 = exp2i(e2);
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
-      const int u = tid + k * kRingConsumers;  // x[8u .. 8u+8): stage u/64, chunk (u%64)/4, word u%4
+      const int u = tid + k * kRingConsumers;  // x[8u .. 8u+8): column u/64, chunk (u%64)/4, word u%4
       if (u < nx) {
         const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
         uint32_t o[4];
@@ -600,116 +664,168 @@ __global__ void __launch_bounds__(kRingThreads, 2)
         xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-    // the last stage's columns past K meet zero codes: their x must be finite
-    for (int u = nx + tid; u < nks * 64; u += kRingConsumers)
+    // the last column's elements past K meet zero codes: their x must be finite
+    for (int u = nx + tid; u < ncols * 64; u += kRingConsumers)
       xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(0, 0, 0, 0);
-  }
-  ring_sync(kRingConsumers);
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may now take the other half
+    ring_sync(kRingConsumers);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may now take the other half
 
-  // lane: rows r0 .. r0+3 of the 120-row stage layout, 16-byte chunk c of each
-  // (rows at or past BR hold stale bytes; their sums are never stored)
-  const int c = tid & (kRingChunks - 1);
-  const int r0 = (tid / kRingChunks) * kRingRows;
-  const uint8_t* lane_codes = ring + r0 * kRingBK + c * 16;
-  const uint8_t* lane_scales = ring + kRingScOff + r0 * kSB + (MX ? c : 2 * c);
-  const uint4* lane_x = xs + c;
-  int slot = 0;
-  uint32_t phase = 0;
-  for (int rb = 0; rb < nb_here; ++rb) {
-    float acc[kRingRows] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int t = 0; t < nks; ++t) {
-      if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&full[slot], phase, kRingWaitNs))) {
-        if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
-        *abort_flag = 1;
-        return;
-      }
-      const uint8_t* pc = lane_codes + slot * kRingStage;
-      const uint8_t* ps = lane_scales + slot * kRingStage;
-      uint4 cw[kRingRows];
-      uint32_t sc[kRingRows];
-#pragma unroll
-      for (int i = 0; i < kRingRows; ++i) {
-        cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingBK);
-        sc[i] = MX ? (uint32_t)ps[i * kSB] : (uint32_t)*reinterpret_cast<const uint16_t*>(ps + i * kSB);
-      }
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[slot]);  // the stage's bytes are in registers
-      if (++slot == S) { slot = 0; phase ^= 1; }
-      const uint4* xp = lane_x + t * 64;
-      float part[kRingRows][2];
-#pragma unroll
-      for (int i = 0; i < kRingRows; ++i) part[i][0] = part[i][1] = 0.0f;
-#pragma unroll
-      for (int wi = 0; wi < 4; ++wi) {  // 8 weights per 32-bit word; words 0-1 block 0, words 2-3 block 1
-        const uint4 xv = xp[wi * 16];
+    // lane: rows slot + 30 i (i < 4, while below BR) of the stage, 16-byte chunk c of each;
+    // the warp's two slots are 2w and 2w + 1, so it skips the i whose even row is past BR
+    const int c = tid & (kRingChunks - 1);
+    const int slot0 = tid / kRingChunks;
+    const int nrow_i = min(kRingRows, (BR - 2 * warp + kRingSlots - 1) / kRingSlots);  // warp-uniform
+    const uint8_t* lane_codes = ring + slot0 * kRingBK + c * 16;
+    const uint8_t* lane_scales = ring + BR * kRingBK + slot0 * kSB + (MX ? c : 2 * c);
+    const uint4* lane_x = xs + c;
+    int sl = 0;
+    uint32_t phase = 0;
+    for (int rb = 0; rb < nb_here && !failed; ++rb) {
+      float acc[kRingRows] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int t = 0; t < ncols; ++t) {
+        if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&full[sl], phase, kRingWaitNs))) {
+          if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+          *abort_flag = 1;
+          failed = true;
+          break;
+        }
+        const uint8_t* pc = lane_codes + sl * SB;
+        const uint8_t* ps = lane_scales + sl * SB;
+        uint4 cw[kRingRows];
+        uint32_t sc[kRingRows];
 #pragma unroll
         for (int i = 0; i < kRingRows; ++i) {
-          const uint32_t word = wi == 0 ? cw[i].x : wi == 1 ? cw[i].y : wi == 2 ? cw[i].z : cw[i].w;
-          float p = part[i][wi >> 1];
-          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
-          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
-          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
-          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
-          part[i][wi >> 1] = p;
+          if (i < nrow_i) {  // rows at or past BR (odd slot of the last i) read stale bytes, never stored
+            cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingSlots * kRingBK);
+            sc[i] = MX ? (uint32_t)ps[i * kRingSlots * kSB]
+                       : (uint32_t)*reinterpret_cast<const uint16_t*>(ps + i * kRingSlots * kSB);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[sl]);  // the stage's bytes are in registers
+        if (++sl == S) { sl = 0; phase ^= 1; }
+        const uint4* xp = lane_x + t * 64;
+        float pt[kRingRows][2];
+#pragma unroll
+        for (int i = 0; i < kRingRows; ++i) pt[i][0] = pt[i][1] = 0.0f;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {  // 8 weights per 32-bit word; words 0-1 block 0, words 2-3 block 1
+          const uint4 xv = xp[wi * 16];
+#pragma unroll
+          for (int i = 0; i < kRingRows; ++i) {
+            if (i < nrow_i) {
+              const uint32_t word = wi == 0 ? cw[i].x : wi == 1 ? cw[i].y : wi == 2 ? cw[i].z : cw[i].w;
+              float p = pt[i][wi >> 1];
+              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
+              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
+              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
+              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
+              pt[i][wi >> 1] = p;
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kRingRows; ++i) {
+          if (i < nrow_i) {
+            if constexpr (MX) {  // one 32-element block per chunk
+              acc[i] = fmaf(pt[i][0] + pt[i][1], e8m0_to_float(sc[i]), acc[i]);
+            } else {
+              const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
+              acc[i] = fmaf(pt[i][0], sf.x, acc[i]);
+              acc[i] = fmaf(pt[i][1], sf.y, acc[i]);
+            }
+          }
         }
       }
+      if (failed) break;
 #pragma unroll
       for (int i = 0; i < kRingRows; ++i) {
-        if constexpr (MX) {  // one 32-element block per chunk
-          acc[i] = fmaf(part[i][0] + part[i][1], e8m0_to_float(sc[i]), acc[i]);
-        } else {
-          const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
-          acc[i] = fmaf(part[i][0], sf.x, acc[i]);
-          acc[i] = fmaf(part[i][1], sf.y, acc[i]);
-        }
+        float v = acc[i];
+#pragma unroll
+        for (int o = kRingChunks / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        acc[i] = v;
+      }
+      if (c < nrow_i) {
+        const float v = c == 0 ? acc[0] : c == 1 ? acc[1] : c == 2 ? acc[2] : acc[3];
+        const int rl = slot0 + kRingSlots * c;
+        if (rl < BR) emit(rb, rl, ldexpf(v * gv, -e));
       }
     }
-#pragma unroll
-    for (int i = 0; i < kRingRows; ++i) {
-      float v = acc[i];
-#pragma unroll
-      for (int o = kRingChunks / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-      acc[i] = v;
-    }
-    if (c < kRingRows) {
-      const float v = c == 0 ? acc[0] : c == 1 ? acc[1] : c == 2 ? acc[2] : acc[3];
-      const int rl = r0 + c;
-      const int row = row_base + rb * BR + rl;
-      if (rl < BR && row < N) {
-        const __nv_bfloat16 o = __float2bfloat16_rn(ldexpf(v * gv, -e));
+  }
+  if (C == 1) return;
+
+  // ---- K split over the cluster: every CTA's partials are in its shared
+  // memory; rank r adds rows [r R / C, (r + 1) R / C) of the R rows over the
+  // ranks in order and stores them.  Every consumer thread passes both
+  // cluster barriers (also after a failed wait: its partials are then NaN),
+  // so no CTA exits while another reads its shared memory.
+  if (failed)
+    for (int i = tid; i < nb_here * BR; i += kRingConsumers) part[i] = __int_as_float(0x7FC00000);
+  ptx::cluster_sync();
+  {
+    const int R = nb_here * BR;
+    const int lo = (int)((int64_t)rank * R / C), hi = (int)((int64_t)(rank + 1) * R / C);
+    for (int r = lo + tid; r < hi; r += kRingConsumers) {
+      float v = ptx::ld_cluster_f32(part + r, 0);
+      for (int j = 1; j < C; ++j) v += ptx::ld_cluster_f32(part + r, (uint32_t)j);
+      const int row = row_base + r;
+      if (row < N) {
+        const __nv_bfloat16 o = __float2bfloat16_rn(v);
         y[row] = *reinterpret_cast<const uint16_t*>(&o);
       }
     }
   }
+  ptx::cluster_sync();
 }
 
 struct RingPlan {
-  int BR, nblk, grid, S;
+  int BR, nblk, grid, S, SB, C;
   size_t smem;
 };
 
-// The ring kernel's shape: rows split evenly over the SMs, shared memory for at
-// least two stages within half of the SM.  False when K does not fit it.
-bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, RingPlan& p) {
+// The ring kernel's shape: split K over C in {1, 2, 4, 8} CTAs of a cluster
+// (forced when force_c != 0), rows split evenly over the SMs' worth of
+// clusters, shared memory for 2..8 stages within half of the SM.  C is the
+// split that gives a CTA the least work (rows x columns; ties to the smaller
+// C).  False when no split fits.
+bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, int force_c, RingPlan& p) {
   // TMA row strides are multiples of 16 bytes: K/16 (NVFP4) or K/32 (MXFP4) scale bytes
-  if (K % (mx ? 512 : 256) != 0 || K > kRingMaxK || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
+  if (K % (mx ? 512 : 256) != 0 || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
   int dev = 0, per_sm = 0, reserved = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
     return false;
-  const int64_t rpc = ((int64_t)num_problems * N + sms - 1) / sms;  // rows of all problems over the SMs
-  p.nblk = (int)((rpc + kRingMaxBR - 1) / kRingMaxBR);
-  p.BR = (int)((rpc + p.nblk - 1) / p.nblk);
-  p.grid = (int)((N + (int64_t)p.nblk * p.BR - 1) / ((int64_t)p.nblk * p.BR));
+  const int kSB = mx ? kRingBK / 16 : kRingBK / 8;
   const int64_t nks = (K / 2 + kRingBK - 1) / kRingBK;
-  const int64_t fixed = nks * 1024 + 256;
   const int64_t budget = per_sm / 2 - reserved;  // two such CTAs per SM
-  if (fixed + 2 * kRingStage > budget) return false;
-  p.S = (int)std::min<int64_t>(4, (budget - fixed) / kRingStage);
-  p.smem = (size_t)(p.S * kRingStage + fixed);
-  return true;
+  bool found = false;
+  int64_t best_work = 0;
+  for (int C = 1; C <= 8; C *= 2) {
+    if (force_c && C != force_c) continue;
+    if ((num_problems > 1 && C > 1) || C > nks) continue;  // grouped calls split rows only
+    const int64_t ncx = (nks + C - 1) / C;
+    if (ncx * 2 * kRingBK > kRingMaxSlice) continue;       // x slice of a CTA
+    const int64_t clusters = std::max<int64_t>(1, sms / C);
+    const int64_t rpc = ((int64_t)num_problems * N + clusters - 1) / clusters;  // rows of all problems over the clusters
+    RingPlan c;
+    c.C = C;
+    c.nblk = (int)((rpc + kRingMaxBR - 1) / kRingMaxBR);
+    c.BR = (int)((rpc + c.nblk - 1) / c.nblk);
+    c.grid = (int)((N + (int64_t)c.nblk * c.BR - 1) / ((int64_t)c.nblk * c.BR)) * C;
+    c.SB = (c.BR * (kRingBK + kSB) + 127) / 128 * 128;
+    const int64_t fixed = ncx * 1024 + 8 * (2 * kRingMaxStages + 1) + 36 * 4 + (int64_t)4 * c.nblk * c.BR + 64;
+    c.S = (int)std::min<int64_t>(kRingMaxStages, (budget - fixed) / c.SB);
+    if (c.S < 2) continue;
+    c.smem = (size_t)(c.S * c.SB + fixed);
+    const int64_t work = (int64_t)c.nblk * c.BR * ncx;
+    if (!found || work < best_work) {
+      p = c;
+      best_work = work;
+      found = true;
+    }
+  }
+  return found;
 }
 
 template <bool MX, bool GROUPED>
@@ -725,13 +841,26 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
                               MX ? kRingBK / 16 : kRingBK / 8, p.BR, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!*encoded) return cudaSuccess;
   static tc::SmemOptIn opt_in;
-  const cudaError_t e = opt_in.ensure((const void*)gemv_ring_kernel<MX, GROUPED>, (int)p.smem);
+  cudaError_t e = opt_in.ensure((const void*)gemv_ring_kernel<MX, GROUPED>, (int)p.smem);
   if (e != cudaSuccess) return e;
-  int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S;
+  int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S, SB = p.SB, C = p.C;
   Problems Pc = P;
-  void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S, &Pc};
-  return tc::launch_pdl((const void*)gemv_ring_kernel<MX, GROUPED>, dim3(p.grid, num_problems), dim3(kRingThreads), p.smem,
-                        stream, args);
+  void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S, &SB, &C, &Pc};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid, num_problems);
+  cfg.blockDim = dim3(kRingThreads);
+  cfg.dynamicSmemBytes = p.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;  // the CTAs that split one row block's K
+  attr[1].val.clusterDim.x = (unsigned)p.C;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.C > 1 ? 2 : 1;
+  return cudaLaunchKernelExC(&cfg, (const void*)gemv_ring_kernel<MX, GROUPED>, args);
 }
 
 }  // namespace
@@ -741,13 +870,14 @@ namespace {
 template <bool MX, bool GROUPED>
 cudaError_t launch_any(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
                        int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream, const Problems& P,
-                       int num_problems) {
+                       int num_problems, int force_splits = 0) {
   RingPlan plan;
-  if (ring_plan(N, K, sms, MX, num_problems, plan)) {
+  if (ring_plan(N, K, sms, MX, num_problems, force_splits > 1 ? force_splits : (force_splits == 1 ? 1 : 0), plan)) {
     bool encoded = false;
     const cudaError_t e = launch_ring<MX, GROUPED>(x, q, s, g, y, N, K, stream, plan, P, num_problems, &encoded);
     if (encoded || e != cudaSuccess) return e;
   }
+  if (force_splits > 1) return cudaErrorInvalidConfiguration;  // the forced split does not fit this shape
   if (MX || K % 32 == 0)
     return launch<8, 16, 2, MX, GROUPED>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
   return launch<8, 8, 2, false, GROUPED>(x, q, s, g, y, (int)N, (int)K, static_weights, stream, P, num_problems);
@@ -758,13 +888,19 @@ const Problems kSingle = {nullptr, nullptr, 1, 1, 0, 0};
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
-                        uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  return launch_any<false, false>(x, q, s, g, y, N, K, sms, static_weights, stream, kSingle, 1);
+                        uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream,
+                        int splits) {
+  return launch_any<false, false>(x, q, s, g, y, N, K, sms, static_weights, stream, kSingle, 1, splits);
 }
 
 cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
-                           int64_t K, int sms, bool static_weights, cudaStream_t stream) {
-  return launch_any<true, false>(x, q, s, nullptr, y, N, K, sms, static_weights, stream, kSingle, 1);
+                           int64_t K, int sms, bool static_weights, cudaStream_t stream, int splits) {
+  return launch_any<true, false>(x, q, s, nullptr, y, N, K, sms, static_weights, stream, kSingle, 1, splits);
+}
+
+bool gemv_split_fits(int64_t N, int64_t K, int sms, bool mx, int splits) {
+  RingPlan plan;
+  return ring_plan(N, K, sms, mx, 1, splits, plan);
 }
 
 cudaError_t launch_gemv_grouped(const uint16_t* X, int64_t ldx, const uint8_t* q, const uint8_t* s,

@@ -17,15 +17,25 @@ cudaError_t launch_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw
                             const float* amax, uint8_t* q, uint8_t* s, float* g_out,
                             cudaStream_t stream, int sms);
 cudaError_t launch_finalize_scale(float* amax_then_g, cudaStream_t stream);
+// Micro-scale search (MSE) quantizer (quantize.cu): the quantize arithmetic with
+// each block's scale chosen among the E4M3 codes within `window` of the
+// round-to-nearest one by the least fp64 squared error.
+cudaError_t launch_quantize_mse(const uint16_t* w, int64_t N, int64_t K, int64_t ldw, const float* amax, int window,
+                                uint8_t* q, uint8_t* s, float* g_out, cudaStream_t stream, int sms);
 // Decode GEMV (gemv.cu).  static_weights: q, s and g are not written by work
 // still running on the stream, so they may be read before it completes
-// (programmatic dependent launch).
+// (programmatic dependent launch).  splits: 0 lets the launcher choose how many
+// CTAs of a cluster split K (1, 2, 4 or 8); a value fixes it, and a split that
+// does not fit the shape returns cudaErrorInvalidConfiguration (1 = no split).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g,
-                        uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream);
+                        uint16_t* y, int64_t N, int64_t K, int sms, bool static_weights, cudaStream_t stream,
+                        int splits = 0);
 // MXFP4 decode GEMV (gemv.cu): one UE8M0 scale per 32 elements, no tensor
 // scale; K a multiple of 32.
 cudaError_t launch_gemv_mx(const uint16_t* x, const uint8_t* q, const uint8_t* s, uint16_t* y, int64_t N,
-                           int64_t K, int sms, bool static_weights, cudaStream_t stream);
+                           int64_t K, int sms, bool static_weights, cudaStream_t stream, int splits = 0);
+// Whether the split-K decode GEMV can run this shape with the given split.
+bool gemv_split_fits(int64_t N, int64_t K, int sms, bool mx, int splits);
 // Grouped (MoE) decode GEMV (gemv.cu): problem p multiplies expert expert_ids[p]
 // of the stacked weights q [E, N, K/2], s [E, N, K/16], g [E] by row
 // token_ids[p] of X [T, K] (leading dimension ldx) into row p of Y (ldy).

@@ -286,6 +286,31 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 namespace nvfp4 {
 namespace ptx {
 
+// ------------------------------------------------------------------ clusters
+
+// This CTA's rank within its thread-block cluster.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every non-exited thread of the cluster arrives, then waits for the others;
+// shared-memory writes before it are visible cluster-wide after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// fp32 at the same shared-memory offset as `local`, in the CTA of the cluster
+// with the given rank (distributed shared memory).
+__device__ __forceinline__ float ld_cluster_f32(const void* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 // 1-D bulk copy global -> shared, completing on `bar` (16-byte aligned
 // addresses, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -82,6 +82,22 @@ typedef enum nvfp4_status {
  */
 #define NVFP4_FLAG_STATIC_WEIGHTS 1u
 
+/*
+ * Decode GEMV only (nvfp4_gemv_ex, mxfp4_gemv_ex): NVFP4_FLAG_KSPLIT(c) with c
+ * in {1, 2, 4, 8} fixes how many CTAs share each block of output rows by
+ * splitting K ("K-parallel" decode GEMV of imp docs/quantization.md, "Dense
+ * layers" pipeline).  The split points fall on 512-element boundaries, so no
+ * 16- or 32-element scale block is cut; the c CTAs form a thread-block cluster
+ * and add their fp32 partial sums in a fixed order through distributed shared
+ * memory (results are deterministic, no workspace).  Without the flag the
+ * library picks c per shape (skinny layers with large K get c > 1).  A c that
+ * does not fit the shape (fewer than c 512-element columns, more than 11520
+ * elements of x per CTA, K not a multiple of 256 / 512 for MXFP4) gives
+ * NVFP4_ERR_SHAPE; c = 1 forbids splitting.
+ */
+#define NVFP4_FLAG_KSPLIT(c) (((uint32_t)(c) & 15u) << 8)
+#define NVFP4_FLAG_KSPLIT_MASK (15u << 8)
+
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 NVFP4_API int nvfp4_version(void);
 
@@ -130,6 +146,28 @@ NVFP4_API nvfp4_status nvfp4_amax(const uint16_t* w, int64_t rows, int64_t cols,
 NVFP4_API nvfp4_status nvfp4_quantize(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
                             const float* amax, uint8_t* q, uint8_t* s, float* g_out,
                             nvfp4_stream_t stream);
+
+/*
+ * Micro-scale search (MSE) quantization (imp docs/quantization.md, micro-scale
+ * search paragraph: each block's FP8 micro-scale chosen by the least
+ * reconstruction error over candidates around the absmax one; measured there
+ * and reverted, kept here as the measured alternative to nvfp4_quantize).
+ * Arguments, layouts, the amax / g_out handling and g are those of
+ * nvfp4_quantize; per 16-block, with c0 the scale byte nvfp4_quantize writes:
+ *   candidates: E4M3 codes c with |c - c0| <= window, clamped to 1..126
+ *     (window 8 = one binade either side; window 0 is nvfp4_quantize);
+ *   each candidate quantizes the block by nvfp4_quantize's element rule with
+ *     d = e4m3(c) * g; its error sum_i (w_i - e2m1(code_i) * d)^2 is formed in
+ *     IEEE fp64, each operation rounded on its own, in index order;
+ *   the least error wins; ties go to the code nearest c0, then to the smaller;
+ *   blocks with c0 == 0 get scale 0 and zero codes.
+ * Output bytes are bit-exact functions of the inputs.  window outside 0..125
+ * gives NVFP4_ERR_INVALID_ARG.  About 17 candidates of fp64 arithmetic per
+ * block: several times the cost of nvfp4_quantize.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize_mse(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                                          const float* amax, int32_t window, uint8_t* q, uint8_t* s,
+                                          float* g_out, nvfp4_stream_t stream);
 
 /*
  * Batch-1 decode GEMV, y[n] = bf16_rn(g * sum_k W_deq[n, k] * x[k]) with fp32

@@ -79,6 +79,33 @@ def test_unknown_flags_rejected():
     assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 0, 64, 1, None) == OK   # N == 0: no-op
 
 
+def test_quantize_mse_validation():
+    """The micro-scale search entry point checks its window, then the same
+    arguments as nvfp4_quantize, before any device work."""
+    assert "nvfp4_quantize_mse" in nv.declared_symbols()
+    for window in (-1, 126, 1000):
+        assert nv.lib.nvfp4_quantize_mse(A, 4, 64, 64, A + 100, window, A + 4096, A + 8192, None, None) == INVALID
+    assert nv.lib.nvfp4_quantize_mse(A, 4, 40, 64, A + 100, 8, A + 4096, A + 8192, None, None) == SHAPE
+    assert nv.lib.nvfp4_quantize_mse(A, 4, 64, 32, A + 100, 8, A + 4096, A + 8192, None, None) == INVALID
+    assert nv.lib.nvfp4_quantize_mse(A, 4, 64, 68, A + 100, 8, A + 4096, A + 8192, None, None) == ALIGN
+    assert nv.lib.nvfp4_quantize_mse(A, 4, 64, 64, None, 8, A + 4096, A + 8192, None, None) == INVALID
+
+
+def test_ksplit_flag_values():
+    """NVFP4_FLAG_KSPLIT(c) takes c in {1, 2, 4, 8} on the GEMV entry points
+    only; anything else is rejected before any device work."""
+    for c in (3, 5, 6, 7, 9, 15):
+        assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 4, 1024, c << 8, None) == INVALID
+        assert nv.lib.mxfp4_gemv_ex(A, A, A, A + 4096, 4, 1024, c << 8, None) == INVALID
+        assert b"KSPLIT" in nv.lib.nvfp4_last_error()
+    for c in (0, 1, 2, 4, 8):
+        assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 0, 1024, c << 8, None) == OK   # N == 0: no-op
+    # the GEMM does not take the GEMV's split flag
+    assert nv.lib.nvfp4_gemm_ex(A, 64, A, A, A, A + 4096, 64, 4, 64, 64, None, 0, 2 << 8, None) == INVALID
+    with pytest.raises(ValueError):
+        nv._ksplit_flag(3)
+
+
 def test_mxfp4_exports_and_validation():
     names = set(nv.declared_symbols())
     assert {"mxfp4_quantize", "mxfp4_gemv", "mxfp4_gemv_ex"} <= names

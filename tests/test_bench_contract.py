@@ -57,3 +57,18 @@ def test_traffic_rows_name_existing_sources():
     for row, files in bench.KERNEL_SOURCES.items():
         for f in files:
             assert os.path.exists(os.path.join(bench.ROOT, f)), (row, f)
+
+
+def test_down_projection_bytes():
+    # the MLP down projection W [5120, 17408]: nibbles + scales + x [17408] + y [5120] + g
+    assert bench.gemv_bytes(5120, 17408) == 44_564_480 + 5_570_560 + 34_816 + 10_240 + 4 == 50_180_100
+
+
+def test_dram_attested_fraction():
+    # measured DRAM bytes per call over the event time, against the HBM peak:
+    # 363.2 MB of quantizer traffic in 66.46 us at a 6542.4 GB/s peak
+    d = bench.dram_attested(363_160_613, 66.46, 6542.4)
+    assert abs(d["GB/s_dram"] - 363_160_613 / 66.46e-6 / 1e9) < 1e-6
+    assert abs(d["frac_hbm_dram"] - d["GB/s_dram"] / 6542.4) < 1e-12
+    assert 0.83 < d["frac_hbm_dram"] < 0.84
+    assert bench.dram_attested(None, 66.46, 6542.4) == {"GB/s_dram": None, "frac_hbm_dram": None}

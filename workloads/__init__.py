@@ -8,7 +8,8 @@ are fed from here.
 Shapes follow a 27B-class decoder layer (hidden 5120, MLP 17408) as used on
 the model card "Qwen3.8-27B-NVFP4 (compressed-tensors)", section
 "Measurements": batch-1 decode, 32-user decode and a 512-token prefill.
-There is no dataset: every tensor is drawn from a fixed seed.
+The MLP down projection of the same layer (N=5120, K=17408) is the skinny
+decode shape.  There is no dataset: every tensor is drawn from a fixed seed.
 
 Recipe (all draws from ``numpy.random.default_rng(seed).spawn(4)``; stream 0
 for W, 1 for the per-row jitter, 2 for the outlier mask, 3 for x):
@@ -51,6 +52,8 @@ CONFIGS = {
                           3 * HIDDEN + 2 * MLP, HIDDEN, 2, "merged"),
     "batch32": LayerConfig("32-user decode GEMM M=32 N=17408 K=5120", 32, MLP, HIDDEN, 3, "layer"),
     "prefill": LayerConfig("prefill GEMM M=512 N=17408 K=5120", 512, MLP, HIDDEN, 4, "layer"),
+    # the MLP down projection of the same layer: few rows, long K (split-K decode GEMV)
+    "down": LayerConfig("down-projection decode GEMV N=5120 K=17408", 1, HIDDEN, MLP, 5, "layer"),
 }
 
 # Relative amax of the five merged members (q, k, v, gate, up): a 3.7x spread,
