@@ -57,8 +57,13 @@ constexpr int kWK = 256;        // k per weight stage (one 128-byte line of code
 // warp about 45 cycles at these N whatever the tile, so one issuer per
 // dequantization group keeps the tensor cores fed), converter, 16 dequantizers.
 constexpr int kProdWarp = 0, kMmaWarp0 = 1, kMmaWarps = 4, kConvWarp = 5, kDeqWarp0 = 6, kDeqWarps = 16;
+// M > 8: one f16-activation producer warp per MMA issuer, so that each
+// issuer's activation tiles are refilled as soon as its own MMAs release them
+// (a single producer serving the four issuers in order made every issuer wait
+// for the slowest one).
+constexpr int kXWarp0 = kDeqWarp0 + kDeqWarps, kXWarps = kMmaWarps;
 constexpr int kMmaWarp = kMmaWarp0;  // also allocates and frees tensor memory
-constexpr int kThreads = (kDeqWarp0 + kDeqWarps) * 32;
+constexpr int kThreads = (kXWarp0 + kXWarps) * 32;
 constexpr int kScanThreads = (1 + kDeqWarps) * 32;  // converter + dequant warps (range scan)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kWideRow = -(1 << 30);
@@ -86,16 +91,20 @@ struct SmallCfg {
   // exact for a consumer that sees every phase of its slot).
   // On the M <= 8 path each dequantization group converts its own B tiles,
   // one per A sub-slot (released together with it).
+  // On the M > 8 path every issuer owns the slots h % kNX of its half
+  // stages h (kNX / 4 of them): 4, 3 and 2 per issuer for N = 16, 32, 64,
+  // enough that a slot's reload (MMA completion, then an L2 round trip) runs
+  // behind the issuer's MMAs on its other slots.
   static constexpr int kXTile = CONV ? 1024 : BNT * 128;
   static constexpr int kXSlot = CONV ? kXTile : 2 * kXTile;
-  static constexpr int kNX = CONV ? 4 * (BNT <= 32 ? 3 : 2) : (BNT <= 32 ? 8 : 4);
+  static constexpr int kNX = CONV ? 4 * (BNT <= 32 ? 3 : 2) : (BNT <= 16 ? 16 : BNT <= 32 ? 12 : 8);
   // +1024: the MMA reads B rows 8..15 one 1024-byte atom past each 8-row tile
   // of the M <= 8 path (those output columns are discarded)
   static constexpr int kXRing = kNX * kXSlot + 1024;
   static constexpr int kWQ = kBM * 128, kWS = kBM * 16, kWStage = kWQ + kWS;
   static constexpr int kBudget = 218 * 1024;
   static constexpr int kWFit = (kBudget - kXRing) / kWStage;
-  static constexpr int kNW = (kWFit > 12 ? 12 : kWFit) / 4 * 4;
+  static constexpr int kNW = (kWFit > 12 ? 12 : kWFit) / 2 * 2;
   // one fp32 accumulator per MMA issuer (summed in the epilogue), then a ring
   // of kNS A sub-slots (64 k of f16 weights = 32 TMEM columns) per
   // dequantization group, so that a group dequantizes the next half stage
@@ -109,7 +118,10 @@ struct SmallCfg {
   static_assert(BNT % 16 == 0 && BNT >= 16 && BNT <= 64, "MMA N");
   static_assert(!CONV || BNT == 16, "the converted path covers M <= 8");
   static_assert(kNW >= 4 && kNW <= 16 && kNX <= 16, "rings");
-  static_assert(kNW % 4 == 0 && kNX % 4 == 0, "slots owned by one group");
+  // a weight stage is read by the groups of its two halves ({0, 1} for even
+  // stages, {2, 3} for odd ones): an even ring keeps each slot with one pair;
+  // an activation slot h % kNX belongs to issuer h % 4
+  static_assert(kNW % 2 == 0 && kNX % 4 == 0, "slots owned by one group");
   static_assert(kABase % 32 == 0 && kABase + 32 * kNA <= (int)kTmemCols, "TMEM columns");
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
@@ -345,6 +357,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mma_commit(&bars->tmem_full);
       if (bars->err) ptx::mbar_wait(&bars->tmem_full, 0, kWaitLimitNs);
     }
+  } else if (warp >= kXWarp0) {
+    // ------------------ M > 8: f16 activation tiles from the pre-pass (TMA), one warp per issuer
+    if constexpr (!CONV) {
+      if (lane == 0) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // written by the pre-pass kernel
+        const int gi = warp - kXWarp0;
+        const int num_h = num_kb / 2;
+        int h = gi;
+        for (; h < num_h; h += kMmaWarps) {  // this issuer's half stages h = gi mod 4, slot h % NX
+          const int xs = h % NX;
+          if (h >= NX && !wait_or_fail(&bars->xempty[xs], ((h / NX) - 1) & 1, bars)) break;
+          ptx::mbar_arrive_expect_tx(&bars->xfull[xs], C::kXSlot);
+#pragma unroll
+          for (int sub = 0; sub < 2; ++sub)
+            ptx::tma_load_2d(xring + xs * C::kXSlot + sub * C::kXTile, &tmap_x, &bars->xfull[xs],
+                             (2 * h + sub) * kBK, m0);
+        }
+        if (bars->err)  // let the copies already issued land before the CTA exits
+          for (int hh = h - NX > gi ? h - NX : gi; hh < h; hh += kMmaWarps)
+            ptx::mbar_wait(&bars->xfull[hh % NX], (hh / NX) & 1, kWaitLimitNs);
+      }
+    }
   } else {
     // ------------------------------- M <= 8: |x| range of every row, all 17 warps
     if constexpr (CONV) {
@@ -379,24 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (CONV) {
         // M <= 8: the dequantization groups convert X themselves
       } else {
-        // ---------------------------------- M > 8: f16 B stages from the pre-pass (TMA)
-        if (lane == 0) {
-          asm volatile("griddepcontrol.wait;" ::: "memory");  // written by the pre-pass kernel
-          int nx = 0;
-          const int num_h = num_kb / 2;
-          for (; nx < num_h; ++nx) {
-            const int xs = nx % NX;
-            if (nx >= NX && !wait_or_fail(&bars->xempty[xs], ((nx / NX) - 1) & 1, bars)) break;
-            ptx::mbar_arrive_expect_tx(&bars->xfull[xs], C::kXSlot);
-#pragma unroll
-            for (int sub = 0; sub < 2; ++sub)
-              ptx::tma_load_2d(xring + xs * C::kXSlot + sub * C::kXTile, &tmap_x, &bars->xfull[xs],
-                               (2 * nx + sub) * kBK, m0);
-          }
-          if (bars->err)
-            for (int wb = nx > NX ? nx - NX : 0; wb < nx; ++wb)
-              ptx::mbar_wait(&bars->xfull[wb % NX], (wb / NX) & 1, kWaitLimitNs);
-        }
+        // M > 8: the activation tiles come from the producer warps kXWarp0.. (one per issuer)
       }
     } else {
       // ------------------------------------------------ dequantize into TMEM

@@ -21,20 +21,27 @@
 //
 // Two kernels:
 //
-// * Ring kernel (K a multiple of 256, K <= 11520): one CTA per SM holding half
-//   of the SM's registers and shared memory, so that the next kernel on the
-//   stream can be resident beside it.  CTA c owns a contiguous range of about
-//   N / #SMs rows.  A producer thread streams the range through a ring of
-//   shared-memory stages with 2-D TMA copies (120 rows x 256 code bytes + their
-//   scales per stage; rows past the end read as zero); 15 consumer warps own
-//   4 rows x one 16-byte chunk per lane, release a stage as soon as its bytes
-//   are in registers, and reduce each row over its 16 lanes once.  After the
-//   previous kernel has finished, x arrives first (one bulk copy), then the
-//   ring, so x is never queued behind weight traffic.  The next kernel on the
-//   stream may start (programmatic dependent launch) once this one has staged
-//   x; its CTAs then wait in the other half of each SM.  The static-weights
-//   flag does not change this kernel: weight requests issued before x, by it
-//   or by the kernel after it, were measured to delay x more than they saved.
+// * Ring kernel (K a multiple of 256): CTAs of half an SM's registers and
+//   shared memory, so that the next kernel on the stream can be resident
+//   beside them.  K may be split over the C in {1, 2, 4, 8} CTAs of a thread-
+//   block cluster ("K-parallel"; each CTA holds at most 11520 elements of x):
+//   each cluster owns a contiguous range of about N / (#SMs / C) rows and rank
+//   r takes its share of the 512-element columns of K.  A producer thread
+//   streams the CTA's range through a ring of shared-memory stages with 2-D
+//   TMA copies (up to 120 rows x 256 code bytes + their scales per stage;
+//   rows past the end read as zero); 15 consumer warps own up to 4 rows x one
+//   16-byte chunk per lane, release a stage as soon as its bytes are in
+//   registers, and reduce each row over its 16 lanes once.  With C > 1 the
+//   CTAs leave fp32 partials in shared memory and the cluster adds them in
+//   rank order through distributed shared memory.  After the previous kernel
+//   has finished, x arrives first (one bulk copy), then the ring, so x is
+//   never queued behind weight traffic.  The next kernel on the stream may
+//   start (programmatic dependent launch) once every CTA of this one has
+//   issued its last stage; its CTAs then wait in the other half of each SM
+//   while this kernel drains.  The static-weights flag does not change this
+//   kernel: weight requests issued before x, into shared memory or into L2,
+//   by it or by the kernel after it, were measured to delay x and the first
+//   stages more than they saved.
 //
 // * Register kernel (every other K): a warp owns R = 8 consecutive rows; lane l
 //   reads the 16-byte chunks l, l+32, ... of each row into two register buffers
@@ -426,6 +433,7 @@ constexpr int kRingRows = 4;                              // rows per lane at mo
 constexpr int kRingMaxBR = kRingSlots * kRingRows;        // 120 rows per stage
 constexpr int kRingMaxSlice = kRingConsumers * 24;        // x elements per CTA: at most 3 uint4 per consumer
 constexpr int kRingMaxStages = 8;
+constexpr int64_t kRingMinInFlight = 64 * 1024;  // ring bytes below which a split of 2 is preferred
 constexpr uint64_t kRingWaitNs = 2000000000ull;
 
 __device__ __forceinline__ void ring_sync(int n) { asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory"); }
@@ -466,6 +474,94 @@ __device__ __noinline__ float dot_exact_range(const uint16_t* __restrict__ x, co
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
   return acc;
+}
+
+// The consumer loop of one warp of the ring kernel: NR rows per lane (a
+// compile-time count, so that the loads, the decode and the FMAs of a stage
+// are straight-line code), rows slot0 + 30 i of each stage, 16-byte chunk c.
+// A warp with NR == 0 only keeps the ring's phases (waits and releases each
+// stage).  emit(rb, local_row, value) receives each row's dot product times
+// g * 2^-e.  Returns false when a bounded wait gave up.
+template <bool MX, int NR, typename Emit>
+__device__ __forceinline__ bool ring_rows(const uint8_t* lane_codes, const uint8_t* lane_scales, const uint4* lane_x,
+                                          uint64_t* full, uint64_t* empty, int S, int SB, int nb_here, int ncols,
+                                          int c, int slot0, int BR, float scale, int e, Emit&& emit) {
+  constexpr int kSB = MX ? kRingBK / 16 : kRingBK / 8;
+  constexpr int R = NR > 0 ? NR : 1;
+  const int lane = threadIdx.x & 31;
+  int sl = 0;
+  uint32_t phase = 0;
+  for (int rb = 0; rb < nb_here; ++rb) {
+    float acc[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) acc[i] = 0.0f;
+    for (int t = 0; t < ncols; ++t) {
+      if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&full[sl], phase, kRingWaitNs))) return false;
+      uint4 cw[R];
+      uint32_t sc[R];
+      if constexpr (NR > 0) {
+        const uint8_t* pc = lane_codes + sl * SB;
+        const uint8_t* ps = lane_scales + sl * SB;
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {  // (the odd slot of the last i may be row BR: stale bytes, never stored)
+          cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingSlots * kRingBK);
+          sc[i] = MX ? (uint32_t)ps[i * kRingSlots * kSB]
+                     : (uint32_t)*reinterpret_cast<const uint16_t*>(ps + i * kRingSlots * kSB);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[sl]);  // the stage's bytes are in registers
+      if (++sl == S) { sl = 0; phase ^= 1; }
+      if constexpr (NR > 0) {
+        const uint4* xp = lane_x + t * 64;
+        float pt[NR][2];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) pt[i][0] = pt[i][1] = 0.0f;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {  // 8 weights per 32-bit word; words 0-1 block 0, words 2-3 block 1
+          const uint4 xv = xp[wi * 16];
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            const uint32_t word = wi == 0 ? cw[i].x : wi == 1 ? cw[i].y : wi == 2 ? cw[i].z : cw[i].w;
+            float p = pt[i][wi >> 1];
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
+            p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
+            pt[i][wi >> 1] = p;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          if constexpr (MX) {  // one 32-element block per chunk
+            acc[i] = fmaf(pt[i][0] + pt[i][1], e8m0_to_float(sc[i]), acc[i]);
+          } else {
+            const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
+            acc[i] = fmaf(pt[i][0], sf.x, acc[i]);
+            acc[i] = fmaf(pt[i][1], sf.y, acc[i]);
+          }
+        }
+      }
+    }
+    if constexpr (NR > 0) {
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        float v = acc[i];
+#pragma unroll
+        for (int o = kRingChunks / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        acc[i] = v;
+      }
+      if (c < NR) {
+        float v = acc[0];
+#pragma unroll
+        for (int i = 1; i < NR; ++i)
+          if (c == i) v = acc[i];
+        const int rl = slot0 + kRingSlots * c;
+        if (rl < BR) emit(rb, rl, ldexpf(v * scale, -e));
+      }
+    }
+  }
+  return true;
 }
 
 // Shared memory: S stages of SB bytes (a stage: BR rows x 256 code bytes, then
@@ -646,7 +742,6 @@ __global__ void __launch_bounds__(kRingThreads, 2)
       const float v = dot_exact_range<MX>(x, q, s, K, row_base + r, k0, k1) * gv;
       if (lane == 0) emit(r / BR, r % BR, v);
     }
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   } else if (!failed) {
     const int e1 = e / 2, e2 = e - e1;  // two exact power-of-two steps
     const float m1 = exp2i(e1), m2 = exp2i(e2);
@@ -668,88 +763,32 @@ __global__ void __launch_bounds__(kRingThreads, 2)
     for (int u = nx + tid; u < ncols * 64; u += kRingConsumers)
       xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(0, 0, 0, 0);
     ring_sync(kRingConsumers);
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may now take the other half
+    // (the next launch is triggered by the producer once it has issued the
+    // CTA's last stage: its CTAs then take the other half of each SM while
+    // this kernel drains its last stages, instead of waiting there for most
+    // of its run)
 
-    // lane: rows slot + 30 i (i < 4, while below BR) of the stage, 16-byte chunk c of each;
-    // the warp's two slots are 2w and 2w + 1, so it skips the i whose even row is past BR
+    // lane: rows slot0 + 30 i (i < NR) of each stage, 16-byte chunk c of each;
+    // the warp's two slots are 2w and 2w + 1, so NR counts the i whose even
+    // row is below BR (warp-uniform; one compiled loop per count)
     const int c = tid & (kRingChunks - 1);
     const int slot0 = tid / kRingChunks;
-    const int nrow_i = min(kRingRows, (BR - 2 * warp + kRingSlots - 1) / kRingSlots);  // warp-uniform
+    const int nrow_i = min(kRingRows, (BR - 2 * warp + kRingSlots - 1) / kRingSlots);
     const uint8_t* lane_codes = ring + slot0 * kRingBK + c * 16;
     const uint8_t* lane_scales = ring + BR * kRingBK + slot0 * kSB + (MX ? c : 2 * c);
     const uint4* lane_x = xs + c;
-    int sl = 0;
-    uint32_t phase = 0;
-    for (int rb = 0; rb < nb_here && !failed; ++rb) {
-      float acc[kRingRows] = {0.0f, 0.0f, 0.0f, 0.0f};
-      for (int t = 0; t < ncols; ++t) {
-        if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&full[sl], phase, kRingWaitNs))) {
-          if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
-          *abort_flag = 1;
-          failed = true;
-          break;
-        }
-        const uint8_t* pc = lane_codes + sl * SB;
-        const uint8_t* ps = lane_scales + sl * SB;
-        uint4 cw[kRingRows];
-        uint32_t sc[kRingRows];
-#pragma unroll
-        for (int i = 0; i < kRingRows; ++i) {
-          if (i < nrow_i) {  // rows at or past BR (odd slot of the last i) read stale bytes, never stored
-            cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingSlots * kRingBK);
-            sc[i] = MX ? (uint32_t)ps[i * kRingSlots * kSB]
-                       : (uint32_t)*reinterpret_cast<const uint16_t*>(ps + i * kRingSlots * kSB);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&empty[sl]);  // the stage's bytes are in registers
-        if (++sl == S) { sl = 0; phase ^= 1; }
-        const uint4* xp = lane_x + t * 64;
-        float pt[kRingRows][2];
-#pragma unroll
-        for (int i = 0; i < kRingRows; ++i) pt[i][0] = pt[i][1] = 0.0f;
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {  // 8 weights per 32-bit word; words 0-1 block 0, words 2-3 block 1
-          const uint4 xv = xp[wi * 16];
-#pragma unroll
-          for (int i = 0; i < kRingRows; ++i) {
-            if (i < nrow_i) {
-              const uint32_t word = wi == 0 ? cw[i].x : wi == 1 ? cw[i].y : wi == 2 ? cw[i].z : cw[i].w;
-              float p = pt[i][wi >> 1];
-              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
-              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
-              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
-              p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
-              pt[i][wi >> 1] = p;
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < kRingRows; ++i) {
-          if (i < nrow_i) {
-            if constexpr (MX) {  // one 32-element block per chunk
-              acc[i] = fmaf(pt[i][0] + pt[i][1], e8m0_to_float(sc[i]), acc[i]);
-            } else {
-              const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
-              acc[i] = fmaf(pt[i][0], sf.x, acc[i]);
-              acc[i] = fmaf(pt[i][1], sf.y, acc[i]);
-            }
-          }
-        }
-      }
-      if (failed) break;
-#pragma unroll
-      for (int i = 0; i < kRingRows; ++i) {
-        float v = acc[i];
-#pragma unroll
-        for (int o = kRingChunks / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-        acc[i] = v;
-      }
-      if (c < nrow_i) {
-        const float v = c == 0 ? acc[0] : c == 1 ? acc[1] : c == 2 ? acc[2] : acc[3];
-        const int rl = slot0 + kRingSlots * c;
-        if (rl < BR) emit(rb, rl, ldexpf(v * gv, -e));
-      }
+    bool ok;
+    switch (nrow_i) {
+      case 4: ok = ring_rows<MX, 4>(lane_codes, lane_scales, lane_x, full, empty, S, SB, nb_here, ncols, c, slot0, BR, gv, e, emit); break;
+      case 3: ok = ring_rows<MX, 3>(lane_codes, lane_scales, lane_x, full, empty, S, SB, nb_here, ncols, c, slot0, BR, gv, e, emit); break;
+      case 2: ok = ring_rows<MX, 2>(lane_codes, lane_scales, lane_x, full, empty, S, SB, nb_here, ncols, c, slot0, BR, gv, e, emit); break;
+      case 1: ok = ring_rows<MX, 1>(lane_codes, lane_scales, lane_x, full, empty, S, SB, nb_here, ncols, c, slot0, BR, gv, e, emit); break;
+      default: ok = ring_rows<MX, 0>(lane_codes, lane_scales, lane_x, full, empty, S, SB, nb_here, ncols, c, slot0, BR, gv, e, emit); break;
+    }
+    if (!ok) {
+      if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+      *abort_flag = 1;
+      failed = true;
     }
   }
   if (C == 1) return;
@@ -785,9 +824,14 @@ struct RingPlan {
 
 // The ring kernel's shape: split K over C in {1, 2, 4, 8} CTAs of a cluster
 // (forced when force_c != 0), rows split evenly over the SMs' worth of
-// clusters, shared memory for 2..8 stages within half of the SM.  C is the
-// split that gives a CTA the least work (rows x columns; ties to the smaller
-// C).  False when no split fits.
+// clusters, shared memory for 2..8 stages within half of the SM.  Without a
+// forced C: no split when it fits and keeps at least 64 KB of weights in
+// flight per CTA, else a split of 2, else the smallest split that fits.  (A
+// sweep of six 5120..17408-row layers on B200: C = 1 is fastest whenever its
+// ring holds 64 KB or more; a short ring (a few rows per CTA) loses to C = 2;
+// C = 4 and 8 were 30-70% slower than C = 2 at equal work per CTA, so they
+// are used only when one CTA's x slice would be too long otherwise.)  False
+// when no split fits.
 bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, int force_c, RingPlan& p) {
   // TMA row strides are multiples of 16 bytes: K/16 (NVFP4) or K/32 (MXFP4) scale bytes
   if (K % (mx ? 512 : 256) != 0 || N < 1 || sms < 1 || N > (int64_t)1 << 30) return false;
@@ -799,9 +843,9 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, int for
   const int kSB = mx ? kRingBK / 16 : kRingBK / 8;
   const int64_t nks = (K / 2 + kRingBK - 1) / kRingBK;
   const int64_t budget = per_sm / 2 - reserved;  // two such CTAs per SM
+  bool fallback_c1 = false;  // (p holds the C = 1 plan when its ring was short)
   bool found = false;
-  int64_t best_work = 0;
-  for (int C = 1; C <= 8; C *= 2) {
+  for (int C = 1; C <= 8 && !found; C *= 2) {
     if (force_c && C != force_c) continue;
     if ((num_problems > 1 && C > 1) || C > nks) continue;  // grouped calls split rows only
     const int64_t ncx = (nks + C - 1) / C;
@@ -818,14 +862,18 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, int for
     c.S = (int)std::min<int64_t>(kRingMaxStages, (budget - fixed) / c.SB);
     if (c.S < 2) continue;
     c.smem = (size_t)(c.S * c.SB + fixed);
-    const int64_t work = (int64_t)c.nblk * c.BR * ncx;
-    if (!found || work < best_work) {
-      p = c;
-      best_work = work;
-      found = true;
+    const bool last_choice = force_c != 0 || C == 8 || (num_problems > 1);
+    if (C == 1 && !last_choice && (int64_t)c.S * c.SB < kRingMinInFlight) {
+      // a short ring: keep it only if no split fits
+      if (!found) p = c;
+      found = false;
+      fallback_c1 = true;
+      continue;
     }
+    p = c;
+    found = true;
   }
-  return found;
+  return found || fallback_c1;
 }
 
 template <bool MX, bool GROUPED>
