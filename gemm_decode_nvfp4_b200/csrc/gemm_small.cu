@@ -74,7 +74,10 @@ constexpr int kEpiBar = 2;       // named barrier of the 16 dequantization warps
 struct SmallBars {
   uint64_t wfull[16], wempty[16];  // weight stage landed / read by the 16 dequant warps
   uint64_t afull[16], aempty[16];  // A sub-slot (group g, slot i at 3g+i) written (128 threads) / read
-  uint64_t xfull[16], xempty[16];  // f16 B tile ready / read by its MMAs
+  uint64_t xfull[16], xempty[16];  // f16 B tile ready / read by its MMAs (xempty: M <= 8 path)
+  // M > 8: the MMAs of group g's k-th 128-k half stage finished (at 4g + k % 4);
+  // frees its two A sub-slots and its B slot with one commit
+  uint64_t hdone[16];
   uint64_t tmem_full;              // every issuer's last MMA finished (4 arrivals)
   uint32_t tmem_addr;
   volatile int err;
@@ -282,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars->xfull[i], CONV ? 32 : 1);
       ptx::mbar_init(&bars->xempty[i], 1);
     }
+    for (int i = 0; i < 16; ++i) ptx::mbar_init(&bars->hdone[i], 1);
     ptx::mbar_init(&bars->tmem_full, kMmaWarps);
     for (int i = 0; i < kConvMaxM; ++i) {
       bars->xmax[i] = 0;
@@ -335,11 +339,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       int sidx = 0;  // 64-k sub-stages of this group so far
       for (int h = gi; h < num_h && !bars->err; h += kMmaWarps) {
         const int xs = h % NX;
-        if (!CONV && !wait_or_fail(&bars->xfull[xs], (h / NX) & 1, bars)) break;
+        if (!CONV) {
+          // one wait for the B tile and one for the half stage's second A
+          // sub-slot: the same 128 threads signal the first sub-slot before
+          // the second, so its phase is complete too (each wait costs this
+          // warp hundreds of cycles, whether or not the phase is complete)
+          if (!wait_or_fail(&bars->xfull[xs], (h / NX) & 1, bars)) break;
+          const int s1 = sidx + 1;
+          if (!wait_or_fail(&bars->afull[gi * C::kNS + s1 % C::kNS], (s1 / C::kNS) & 1, bars)) break;
+        }
 #pragma unroll
         for (int sub = 0; sub < 2; ++sub, ++sidx) {
           const int slot = gi * C::kNS + sidx % C::kNS;
-          if (!wait_or_fail(&bars->afull[slot], (sidx / C::kNS) & 1, bars)) break;
+          if (CONV && !wait_or_fail(&bars->afull[slot], (sidx / C::kNS) & 1, bars)) break;
           ptx::tc_fence_after();
           const uint32_t a_col = tmem + (uint32_t)(C::kABase + 32 * slot);
           const uint32_t b_tile = CONV ? ptx::smem_u32(xring + slot * C::kXSlot)
@@ -348,9 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < kBK / 16; ++j)  // the issuer's first MMA overwrites its accumulator
             ptx::mma_ts_f16(d_acc, a_col + 8 * j, ptx::sw128_kmajor_desc(b_tile + 32 * j), C::kIdesc,
                             h != gi || sub != 0 || j != 0);
-          ptx::mma_commit(&bars->aempty[slot]);
+          if (CONV) ptx::mma_commit(&bars->aempty[slot]);
         }
-        if (!CONV) ptx::mma_commit(&bars->xempty[xs]);
+        // M > 8: one commit frees both A sub-slots and the B slot of the half stage
+        if (!CONV) ptx::mma_commit(&bars->hdone[gi * 4 + ((h - gi) / kMmaWarps) % 4]);
       }
       // arrives when every MMA of this issuer is done (also on the error path,
       // so that TMEM is never freed under a running MMA)
@@ -367,7 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int h = gi;
         for (; h < num_h; h += kMmaWarps) {  // this issuer's half stages h = gi mod 4, slot h % NX
           const int xs = h % NX;
-          if (h >= NX && !wait_or_fail(&bars->xempty[xs], ((h / NX) - 1) & 1, bars)) break;
+          // the slot was last read by this issuer's half stage kk - NX / 4 (kk = its index among them)
+          const int kk = (h - gi) / kMmaWarps, kprev = kk - NX / kMmaWarps;
+          if (kprev >= 0 && !wait_or_fail(&bars->hdone[gi * 4 + kprev % 4], (kprev / 4) & 1, bars)) break;
           ptx::mbar_arrive_expect_tx(&bars->xfull[xs], C::kXSlot);
 #pragma unroll
           for (int sub = 0; sub < 2; ++sub)
@@ -470,8 +485,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           dequant8(c1.y, __byte_perm(s23, 0, 0x1010), v + 20);
           dequant8(c1.z, __byte_perm(s23, 0, 0x3232), v + 24);
           dequant8(c1.w, __byte_perm(s23, 0, 0x3232), v + 28);
-          // the sub-slot is free once the MMAs of its previous use finished
-          if (round > 0 && !__all_sync(0xFFFFFFFFu, wait_or_fail(&bars->aempty[slot], (round - 1) & 1, bars))) {
+          // the sub-slot is free once the MMAs of its previous use (sub-stage
+          // sidx - kNS) finished: for M > 8 that is the group's half stage
+          // (sidx - kNS) / 2, whose MMAs signal hdone with one commit
+          const int kprev = (sidx - C::kNS) / 2;
+          if (round > 0 && !__all_sync(0xFFFFFFFFu,
+                                       CONV ? wait_or_fail(&bars->aempty[slot], (round - 1) & 1, bars)
+                                            : wait_or_fail(&bars->hdone[grp * 4 + kprev % 4], (kprev / 4) & 1, bars))) {
             ok = false;
             break;
           }
