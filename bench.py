@@ -75,6 +75,7 @@ MSE_FP64_OPS_PER_CANDIDATE = 64  # 16 elements x (multiply, subtract, square, ad
 FP4_PER_BF16 = 4  # nominal dense FP4 / BF16 tensor throughput of B200 (9 / 2.25 PFLOP/s)
 
 MOE = {"E": 128, "N": 1536, "K": 2048, "top": 8}  # synthetic MoE layer: stacked experts, top-8 routing, one token
+MOE_T = 4  # tokens per call of the multi-token grouped row
 
 
 def moe_bytes(n_problems: int, N: int, K: int) -> int:
@@ -114,6 +115,7 @@ KERNEL_SOURCES = {
     "mx_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "mx_quantize": [_CSRC + "quantize.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh"],
     "moe_gemv": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "moe_gemv_t4": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "gemv_down": [_CSRC + "gemv.cu", _CSRC + "nvfp4_device.cuh", _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "w4a4_m512": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
                   _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
@@ -323,6 +325,19 @@ def run_gpu(args):
         for i in range(copies):
             nv.gemv_grouped(moe_x, moe_q, moe_s, moe_g, moe_ids[i], moe_tok, moe_y)
 
+    # the same layer with MOE_T tokens per call (each to its own top-8 experts):
+    # one launch covers MOE_T * 8 problems, amortising the dependent-launch cost
+    gen = torch.Generator().manual_seed(5)
+    moe_ids_t = torch.stack([torch.cat([torch.randperm(me, generator=gen)[:mtop] for _ in range(MOE_T)])
+                             for _ in range(copies)]).to(torch.int32).to(dev)
+    moe_tok_t = torch.arange(MOE_T, dtype=torch.int32).repeat_interleave(mtop).to(dev)
+    moe_x_t = workloads.activations(MOE_T, mk, 6).to(dev)
+    moe_y_t = torch.empty((MOE_T * mtop, mn), dtype=torch.bfloat16, device=dev)
+
+    def moe_t_all():
+        for i in range(copies):
+            nv.gemv_grouped(moe_x_t, moe_q, moe_s, moe_g, moe_ids_t[i], moe_tok_t, moe_y_t)
+
     # MLP down projection of the same layer, W [5120, 17408]: few rows, long K,
     # the split-K decode GEMV (the library's choice of split), 8 copies (400 MB)
     dcfg = workloads.CONFIGS["down"]
@@ -384,6 +399,7 @@ def run_gpu(args):
         rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
     rows.append(("mx_gemv", mx_gemv_all, copies, 1))
     rows.append(("moe_gemv", moe_all, copies, 1))
+    rows.append(("moe_gemv_t4", moe_t_all, copies, 1))
     rows.append(("gemv_down", gemv_down_all, copies, 1))
     rows.append(("gemv_ordered", gemv_ordered_all, copies, 1))
     rows.append(("gemv", gemv_all, copies, 1))
@@ -499,6 +515,14 @@ def run_gpu(args):
             "fp64_ops_per_block_max": MSE_FP64_OPS_PER_CANDIDATE * (2 * MSE_WINDOW + 1),
             "what": "amax + micro-scale search quantizer (E4M3 candidates within 8 codes, fp64 error): "
                     "FP64-bound; the pages report about 6x the round-to-nearest cost"}
+    if "moe_gemv_t4" in per_launch_ms:
+        P = MOE_T * MOE["top"]
+        mb = moe_bytes(P, MOE["N"], MOE["K"]) + 2 * MOE["K"] * (MOE_T - 1)
+        mg = mb / (per_launch_ms["moe_gemv_t4"] * 1e-3) / 1e9
+        kernels["moe_gemv_t4"] = {"us": per_launch_ms["moe_gemv_t4"] * 1e3, "GB/s": mg, "frac_hbm": mg / hbm, "bytes": mb,
+                                  "us_per_token": per_launch_ms["moe_gemv_t4"] * 1e3 / MOE_T,
+                                  "workload": f"grouped decode GEMV: {MOE_T} tokens x top-{MOE['top']} of {MOE['E']} "
+                                              f"stacked experts [{MOE['N']}, {MOE['K']}] = {P} problems per launch"}
     if "gemv_down" in per_launch_ms:
         db = gemv_bytes(dcfg.N, dcfg.K)
         dgbs = db / (per_launch_ms["gemv_down"] * 1e-3) / 1e9
@@ -590,9 +614,9 @@ def run_gpu(args):
             "config": {"workload": WORKLOAD, "N": N, "K": K, "M": 1, "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2: {copies} rotating weight copies "
                              f"({copies * (N * K // 2 + N * K // 16) / 1e6:.0f} MB) per graph",
-                       "row_order": "quantize, MSE quantize, MXFP4 quantize (each followed by an untimed read of 2 x L2 that writes back their dirty output), gemm M=512, W4A4 M=512 (step), W4A4 GEMM, gemm M=32, MXFP4 gemv, MoE gemv, down-projection gemv, gemv ordered, gemv static: each GEMV graph "
+                       "row_order": "quantize, MSE quantize, MXFP4 quantize (each followed by an untimed read of 2 x L2 that writes back their dirty output), gemm M=512, W4A4 M=512 (step), W4A4 GEMM, gemm M=32, MXFP4 gemv, MoE gemv (1 and 4 tokens), down-projection gemv, gemv ordered, gemv static: each GEMV graph "
                                     "follows GEMVs, not the rows that leave tens of MB of dirty output in L2",
-                       "step": "quantize [17408,5120] (NVFP4 round-to-nearest, NVFP4 micro-scale search, MXFP4) + gemm M=512 + W4A4 M=512 (quantize X + GEMM) + W4A4 GEMM + gemm M=32 + MXFP4 gemv + grouped MoE gemv + down-projection gemv [5120, 17408] (split-K) + gemv M=1 (x2: ordered and static-weights)",
+                       "step": "quantize [17408,5120] (NVFP4 round-to-nearest, NVFP4 micro-scale search, MXFP4) + gemm M=512 + W4A4 M=512 (quantize X + GEMM) + W4A4 GEMM + gemm M=32 + MXFP4 gemv + grouped MoE gemv (1 and 4 tokens) + down-projection gemv [5120, 17408] (split-K) + gemv M=1 (x2: ordered and static-weights)",
             "gemv_launch": "8 GEMVs per graph on 8 weight copies, programmatic dependent launch (static weights)"},
             "roofline": {"bound": "hbm", "achieved": gemv_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": gemv_gbs / hbm, "traffic": traffic,
@@ -688,7 +712,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "quantize_mse", "gemm_m32",
                                                       "gemm_m512", "mx_gemv", "mx_quantize", "moe_gemv",
-                                                      "gemv_down", "w4a4_m512", "w4a4_gemm"],
+                                                      "gemv_down", "moe_gemv_t4", "w4a4_m512", "w4a4_gemm"],
                     help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps

@@ -41,7 +41,11 @@
 //   while this kernel drains.  The static-weights flag does not change this
 //   kernel: weight requests issued before x, into shared memory or into L2,
 //   by it or by the kernel after it, were measured to delay x and the first
-//   stages more than they saved.
+//   stages more than they saved.  One unsplit problem with full row blocks
+//   (90-120 rows) runs a specialised copy with a fixed stage layout and four
+//   consecutive rows per lane, which was measured faster on those shapes; it
+//   requests its first stage before the dependency wait when the weights are
+//   static (one stage gained, more lost).
 //
 // * Register kernel (every other K): a warp owns R = 8 consecutive rows; lane l
 //   reads the 16-byte chunks l, l+32, ... of each row into two register buffers
@@ -817,9 +821,251 @@ __global__ void __launch_bounds__(kRingThreads, 2)
   ptx::cluster_sync();
 }
 
+// The same ring for one unsplit problem with rows of at least 90 per block:
+// a fixed 120-row stage layout and 4 consecutive rows per lane (every lane's
+// rows are valid, so no per-warp row counts).  Measured faster on the
+// 17408-row decode layer than the general kernel above (10.4 against
+// 10.9 µs per launch in one process on one B200); the general kernel serves
+// split-K, grouped and short-row launches.  With static weights the first
+// stage is requested before the dependency wait.
+constexpr int kRing1ScOff = kRingMaxBR * kRingBK;                      // scales after a fixed 120-row code block
+constexpr int kRing1Stage = kRing1ScOff + kRingMaxBR * (kRingBK / 8);  // 34560 bytes
+constexpr int kRing1MinBR = 90;                                        // rows per block the kernel is used from
+
+template <bool MX>
+__global__ void __launch_bounds__(kRingThreads, 2)
+    gemv_ring1_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap ts,
+                     const uint16_t* __restrict__ x, const uint8_t* __restrict__ q, const uint8_t* __restrict__ s,
+                     const float* __restrict__ g, uint16_t* __restrict__ y, int N, int K, int BR, int nblk,
+                     int S, int static_w) {
+  extern __shared__ __align__(1024) uint8_t sm[];
+  constexpr int kSB = MX ? kRingBK / 16 : kRingBK / 8;  // scale bytes of a row per stage
+  const int nks = (K / 2 + kRingBK - 1) / kRingBK;  // stages per row block
+  uint8_t* ring = sm;
+  uint4* xs = reinterpret_cast<uint4*>(sm + S * kRing1Stage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(xs + nks * 64);
+  uint64_t* empty = full + S;
+  uint64_t* xfull = empty + S;
+  uint32_t* red = reinterpret_cast<uint32_t*>(xfull + 1);        // [2][16]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red + 32);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row_base = blockIdx.x * nblk * BR;
+  const int nb_here = min(nblk, (N - row_base + BR - 1) / BR);
+  const int total = nb_here * nks;
+
+  if (tid == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kRingConsumerWarps);
+    }
+    ptx::mbar_init(xfull, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kRingConsumerWarps) {  // ------------------------------------------------- producer
+    if (lane != 0) return;
+    ptx::prefetch_tmap(&tq);
+    ptx::prefetch_tmap(&ts);
+    uint64_t policy;  // each weight byte is read once: do not keep it in L2
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+    int n = 0, slot = 0, t = 0, rb = 0, e_id = 0;
+    uint32_t phase = 0;
+    auto issue = [&]() {
+      uint8_t* dst = ring + slot * kRing1Stage;
+      const int row0 = row_base + rb * BR;
+      ptx::mbar_arrive_expect_tx(&full[slot], (uint32_t)BR * (kRingBK + kSB));
+      tma_load_3d_evict_first(dst, &tq, &full[slot], t * kRingBK, row0, e_id, policy);
+      tma_load_3d_evict_first(dst + kRing1ScOff, &ts, &full[slot], t * kSB, row0, e_id, policy);
+      if (++slot == S) { slot = 0; phase ^= 1; }
+      if (++t == nks) { t = 0; ++rb; }
+    };
+    // static weights: the first stage is requested before the previous kernel
+    // has finished (one stage: more delayed x and the running kernel's stream)
+    if (static_w && total > 0) {
+      issue();
+      ++n;
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x (and, without static weights, the weights) only after this
+    ptx::mbar_arrive_expect_tx(xfull, (uint32_t)K * 2);
+    ptx::bulk_load(xs, x, (uint32_t)K * 2, xfull);
+    for (; n < total; ++n) {
+      if (n >= S) {  // wait until the consumers have released this slot (or have given up on the ring)
+        bool ok = ptx::mbar_try_wait(&empty[slot], phase ^ 1);
+        const uint64_t t0 = ok ? 0 : ptx::globaltimer_ns();
+        while (!ok && !*abort_flag) {
+          if (ptx::globaltimer_ns() - t0 > kRingWaitNs) {
+            atomicAdd(&g_gemv_wait_timeouts, 1u);
+            break;
+          }
+          ok = ptx::mbar_try_wait(&empty[slot], phase ^ 1);
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) break;
+      issue();
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // nothing may still be landing in shared memory when the CTA exits
+    for (int m = max(0, n - S); m < n; ++m) ptx::mbar_wait(&full[m % S], (m / S) & 1, kRingWaitNs);
+    ptx::mbar_wait(xfull, 0, kRingWaitNs);
+    return;
+  }
+
+  // ------------------------------------------------------------------------------- consumers
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // y is written only after the previous kernel
+  if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(xfull, 0, kRingWaitNs))) {
+    if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+    *abort_flag = 1;
+    return;
+  }
+  // range of |x| over the raw BF16 bit patterns, which stay in registers
+  const int nx = K >> 3;
+  uint4 raw[3];
+  uint32_t mx = 0, mn = 0xFFFFu;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int u = tid + k * kRingConsumers;
+    raw[k] = u < nx ? xs[u] : make_uint4(0, 0, 0, 0);
+    const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = w4[j] & 0x7FFFu, hi = (w4[j] >> 16) & 0x7FFFu;
+      mx = max(mx, max(lo, hi));
+      mn = min(mn, min(lo ? lo : 0xFFFFu, hi ? hi : 0xFFFFu));
+    }
+  }
+  mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+  mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+  if (lane == 0) { red[warp] = mx; red[16 + warp] = mn; }
+  ring_sync(kRingConsumers);  // every raw value is in registers: the buffer may be overwritten
+  mx = red[0]; mn = red[16];
+#pragma unroll
+  for (int w = 1; w < kRingConsumerWarps; ++w) { mx = max(mx, red[w]); mn = min(mn, red[16 + w]); }
+  bool fast = true;
+  int e = 0;
+  if (mx >= 0x7F80u) {
+    fast = false;
+  } else if (mx != 0) {
+    const int hi_exp = bf16_ilogb(mx), lo_exp = bf16_ilogb(mn);
+    e = 15 - hi_exp;
+    fast = hi_exp - lo_exp <= 32;
+  }
+  const float gv = MX ? 1.0f : *g;
+  if (!fast) {  // x outside the f16 window: the producer stops, every warp takes rows exactly
+    *abort_flag = 1;
+    const int nrows = min(N - row_base, nblk * BR);
+    for (int r = warp; r < nrows; r += kRingConsumerWarps) rows_exact<MX>(x, q, s, g, y, N, K, row_base + r, 1);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    return;
+  }
+  {
+    const int e1 = e / 2, e2 = e - e1;  // two exact power-of-two steps
+    const float m1 = exp2i(e1), m2 = exp2i(e2);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const int u = tid + k * kRingConsumers;  // x[8u .. 8u+8): stage u/64, chunk (u%64)/4, word u%4
+      if (u < nx) {
+        const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = __floats2half2_rn(bf16lo_to_float(w4[j]) * m1 * m2, bf16hi_to_float(w4[j]) * m1 * m2);
+          o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    // the last stage's columns past K meet zero codes: their x must be finite
+    for (int u = nx + tid; u < nks * 64; u += kRingConsumers)
+      xs[(u >> 6) * 64 + (u & 3) * 16 + ((u & 63) >> 2)] = make_uint4(0, 0, 0, 0);
+  }
+  ring_sync(kRingConsumers);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // the next kernel may now take the other half
+
+  // lane: rows r0 .. r0+3 of the 120-row stage layout, 16-byte chunk c of each
+  // (rows at or past BR hold stale bytes; their sums are never stored)
+  const int c = tid & (kRingChunks - 1);
+  const int r0 = (tid / kRingChunks) * kRingRows;
+  const uint8_t* lane_codes = ring + r0 * kRingBK + c * 16;
+  const uint8_t* lane_scales = ring + kRing1ScOff + r0 * kSB + (MX ? c : 2 * c);
+  const uint4* lane_x = xs + c;
+  int slot = 0;
+  uint32_t phase = 0;
+  for (int rb = 0; rb < nb_here; ++rb) {
+    float acc[kRingRows] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int t = 0; t < nks; ++t) {
+      if (!__all_sync(0xFFFFFFFFu, ptx::mbar_wait(&full[slot], phase, kRingWaitNs))) {
+        if (lane == 0) atomicAdd(&g_gemv_wait_timeouts, 1u);
+        *abort_flag = 1;
+        return;
+      }
+      const uint8_t* pc = lane_codes + slot * kRing1Stage;
+      const uint8_t* ps = lane_scales + slot * kRing1Stage;
+      uint4 cw[kRingRows];
+      uint32_t sc[kRingRows];
+#pragma unroll
+      for (int i = 0; i < kRingRows; ++i) {
+        cw[i] = *reinterpret_cast<const uint4*>(pc + i * kRingBK);
+        sc[i] = MX ? (uint32_t)ps[i * kSB] : (uint32_t)*reinterpret_cast<const uint16_t*>(ps + i * kSB);
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[slot]);  // the stage's bytes are in registers
+      if (++slot == S) { slot = 0; phase ^= 1; }
+      const uint4* xp = lane_x + t * 64;
+      float part[kRingRows][2];
+#pragma unroll
+      for (int i = 0; i < kRingRows; ++i) part[i][0] = part[i][1] = 0.0f;
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {  // 8 weights per 32-bit word; words 0-1 block 0, words 2-3 block 1
+        const uint4 xv = xp[wi * 16];
+#pragma unroll
+        for (int i = 0; i < kRingRows; ++i) {
+          const uint32_t word = wi == 0 ? cw[i].x : wi == 1 ? cw[i].y : wi == 2 ? cw[i].z : cw[i].w;
+          float p = part[i][wi >> 1];
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<0>(word), xv.x, p);
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<1>(word), xv.y, p);
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<2>(word), xv.z, p);
+          p = fma2_f16_f32(e2m1x2_byte_to_f16x2<3>(word), xv.w, p);
+          part[i][wi >> 1] = p;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kRingRows; ++i) {
+        if constexpr (MX) {  // one 32-element block per chunk
+          acc[i] = fmaf(part[i][0] + part[i][1], e8m0_to_float(sc[i]), acc[i]);
+        } else {
+          const float2 sf = f16x2_to_float2(e4m3x2_to_f16x2(sc[i]));
+          acc[i] = fmaf(part[i][0], sf.x, acc[i]);
+          acc[i] = fmaf(part[i][1], sf.y, acc[i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kRingRows; ++i) {
+      float v = acc[i];
+#pragma unroll
+      for (int o = kRingChunks / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+      acc[i] = v;
+    }
+    if (c < kRingRows) {
+      const float v = c == 0 ? acc[0] : c == 1 ? acc[1] : c == 2 ? acc[2] : acc[3];
+      const int rl = r0 + c;
+      const int row = row_base + rb * BR + rl;
+      if (rl < BR && row < N) {
+        const __nv_bfloat16 o = __float2bfloat16_rn(ldexpf(v * gv, -e));
+        y[row] = *reinterpret_cast<const uint16_t*>(&o);
+      }
+    }
+  }
+}
+
 struct RingPlan {
   int BR, nblk, grid, S, SB, C;
   size_t smem;
+  int64_t budget;  // shared memory a CTA may take (half of the SM)
 };
 
 // The ring kernel's shape: split K over C in {1, 2, 4, 8} CTAs of a cluster
@@ -854,6 +1100,7 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, int for
     const int64_t rpc = ((int64_t)num_problems * N + clusters - 1) / clusters;  // rows of all problems over the clusters
     RingPlan c;
     c.C = C;
+    c.budget = budget;
     c.nblk = (int)((rpc + kRingMaxBR - 1) / kRingMaxBR);
     c.BR = (int)((rpc + c.nblk - 1) / c.nblk);
     c.grid = (int)((N + (int64_t)c.nblk * c.BR - 1) / ((int64_t)c.nblk * c.BR)) * C;
@@ -879,7 +1126,7 @@ bool ring_plan(int64_t N, int64_t K, int sms, bool mx, int num_problems, int for
 template <bool MX, bool GROUPED>
 cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, const float* g, uint16_t* y,
                         int64_t N, int64_t K, cudaStream_t stream, const RingPlan& p, const Problems& P,
-                        int num_problems, bool* encoded) {
+                        int num_problems, bool static_weights, bool* encoded) {
   CUtensorMap tq, ts;  // [E, N, K/2] codes and [E, N, scale bytes]: the expert is the third coordinate
   const int64_t sbytes = MX ? K / 32 : K / 16;  // scale bytes per row
   const int64_t E = P.expert_ids ? P.E : 1;
@@ -888,10 +1135,24 @@ cudaError_t launch_ring(const uint16_t* x, const uint8_t* q, const uint8_t* s, c
              tc::make_tmap_3d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, s, sbytes, N, E, sbytes, N * sbytes,
                               MX ? kRingBK / 16 : kRingBK / 8, p.BR, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!*encoded) return cudaSuccess;
+  int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S, SB = p.SB, C = p.C;
+  if (!GROUPED && p.C == 1 && p.BR >= kRing1MinBR) {  // one unsplit problem with full row blocks
+    const int64_t nks = (K / 2 + kRingBK - 1) / kRingBK;
+    const int64_t fixed = nks * 1024 + 256;
+    const int S1 = (int)std::min<int64_t>(4, (p.budget - fixed) / kRing1Stage);
+    if (S1 >= 2) {
+      const size_t smem1 = (size_t)(S1 * kRing1Stage + fixed);
+      static tc::SmemOptIn opt_in1;
+      cudaError_t e = opt_in1.ensure((const void*)gemv_ring1_kernel<MX>, (int)smem1);
+      if (e != cudaSuccess) return e;
+      int S1v = S1, sw = static_weights ? 1 : 0;
+      void* args1[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S1v, &sw};
+      return tc::launch_pdl((const void*)gemv_ring1_kernel<MX>, dim3(p.grid), dim3(kRingThreads), smem1, stream, args1);
+    }
+  }
   static tc::SmemOptIn opt_in;
   cudaError_t e = opt_in.ensure((const void*)gemv_ring_kernel<MX, GROUPED>, (int)p.smem);
   if (e != cudaSuccess) return e;
-  int Ni = (int)N, Ki = (int)K, BR = p.BR, nblk = p.nblk, S = p.S, SB = p.SB, C = p.C;
   Problems Pc = P;
   void* args[] = {&tq, &ts, &x, &q, &s, &g, &y, &Ni, &Ki, &BR, &nblk, &S, &SB, &C, &Pc};
   cudaLaunchConfig_t cfg = {};
@@ -922,7 +1183,8 @@ cudaError_t launch_any(const uint16_t* x, const uint8_t* q, const uint8_t* s, co
   RingPlan plan;
   if (ring_plan(N, K, sms, MX, num_problems, force_splits > 1 ? force_splits : (force_splits == 1 ? 1 : 0), plan)) {
     bool encoded = false;
-    const cudaError_t e = launch_ring<MX, GROUPED>(x, q, s, g, y, N, K, stream, plan, P, num_problems, &encoded);
+    const cudaError_t e =
+        launch_ring<MX, GROUPED>(x, q, s, g, y, N, K, stream, plan, P, num_problems, static_weights, &encoded);
     if (encoded || e != cudaSuccess) return e;
   }
   if (force_splits > 1) return cudaErrorInvalidConfiguration;  // the forced split does not fit this shape

@@ -72,3 +72,10 @@ def test_dram_attested_fraction():
     assert abs(d["frac_hbm_dram"] - d["GB/s_dram"] / 6542.4) < 1e-12
     assert 0.83 < d["frac_hbm_dram"] < 0.84
     assert bench.dram_attested(None, 66.46, 6542.4) == {"GB/s_dram": None, "frac_hbm_dram": None}
+
+
+def test_moe_multi_token_bytes():
+    # 4 tokens x top-8: 32 problems' expert weights + y rows + ids and g, and the 4 token rows of x
+    P = bench.MOE_T * bench.MOE["top"]
+    e = 1536 * 2048 // 2 + 1536 * 2048 // 16
+    assert bench.moe_bytes(P, 1536, 2048) + 2 * 2048 * (bench.MOE_T - 1) == P * (e + 2 * 1536 + 8 + 4) + 2 * 2048 * bench.MOE_T
