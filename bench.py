@@ -121,6 +121,8 @@ KERNEL_SOURCES = {
                   _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
     "w4a4_gemm": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
                   _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
+    "w4a4_pair": [_CSRC + "gemm_w4a4.cu", _CSRC + "nvfp4_quant.cuh", _CSRC + "nvfp4_device.cuh",
+                  _CSRC + "sm100_ptx.cuh", _CSRC + "tc_host.h"],
 }
 
 
@@ -363,7 +365,7 @@ def run_gpu(args):
 
     # W4A4 prefill (NVFP4 activations): the same 8 weight copies, scales
     # rearranged once for the block-scaled tensor cores
-    w4_ok = args.only in ("all", "w4a4_m512", "w4a4_gemm")
+    w4_ok = args.only in ("all", "w4a4_m512", "w4a4_gemm", "w4a4_pair")
     if w4_ok:
         smmas = [nv.w4a4_prepare_weights(ss[i], K) for i in range(copies)]
         ws_w4 = torch.empty((nv.w4a4_workspace_size(512, K),), dtype=torch.uint8, device=dev)
@@ -378,6 +380,10 @@ def run_gpu(args):
         def w4a4_gemm_all():  # the GEMM kernel alone on quantized activations
             for i in range(copies):
                 nv.w4a4_gemm(w4_qx, w4_sx, w4_amax, qs[i], smmas[i], g0, Y512w, static_weights=True)
+
+        def w4a4_pair_all():  # the same GEMM on tiles of 256 weight rows over pairs of SMs
+            for i in range(copies):
+                nv.w4a4_gemm(w4_qx, w4_sx, w4_amax, qs[i], smmas[i], g0, Y512w, static_weights=True, pair=True)
 
     rows.append(("quantize", quant_all, 1, 2))
     rows.append(("quantize_mse", quant_mse_all, 1, 2))
@@ -395,6 +401,7 @@ def run_gpu(args):
     if w4_ok:
         rows.append(("w4a4_m512", w4a4_all, copies, 3))  # amax + quantize X + GEMM per call
         rows.append(("w4a4_gemm", w4a4_gemm_all, copies, 1))
+        rows.append(("w4a4_pair", w4a4_pair_all, copies, 1))
     if gemm_ok:
         rows.append(("gemm_m32", m32_all, copies, 2))    # X prep + GEMM per call
     rows.append(("mx_gemv", mx_gemv_all, copies, 1))
@@ -547,7 +554,7 @@ def run_gpu(args):
             kernels[name] = {"unavailable": gemm_err}
 
     fp4_peak = bf16_burst * FP4_PER_BF16
-    for name in ("w4a4_m512", "w4a4_gemm"):
+    for name in ("w4a4_m512", "w4a4_gemm", "w4a4_pair"):
         if name in per_launch_ms:
             t = per_launch_ms[name] * 1e-3
             fl = 2.0 * 512 * N * K
@@ -557,7 +564,8 @@ def run_gpu(args):
                              "fp4_peak_source": f"{peaks['source']} bf16 x {FP4_PER_BF16} (nominal dense FP4/BF16)",
                              "GB/s": byt / t / 1e9, "frac_hbm": byt / t / 1e9 / hbm, "bytes": byt,
                              "what": ("activation amax + NVFP4 quantize of X + block-scaled FP4 GEMM"
-                                      if name == "w4a4_m512" else "block-scaled FP4 GEMM on quantized X")}
+                                      if name == "w4a4_m512" else "block-scaled FP4 GEMM on quantized X"
+                                      + (", tiles of 256 weight rows on pairs of SMs" if name == "w4a4_pair" else ""))}
 
     # ---- end to end through the public API with host buffers (decode GEMV):
     # pinned x -> device, GEMV, y -> pinned host, every step.
@@ -712,7 +720,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default="all", choices=["all", "gemv", "gemv_ordered", "quantize", "quantize_mse", "gemm_m32",
                                                       "gemm_m512", "mx_gemv", "mx_quantize", "moe_gemv",
-                                                      "gemv_down", "moe_gemv_t4", "w4a4_m512", "w4a4_gemm"],
+                                                      "gemv_down", "moe_gemv_t4", "w4a4_m512", "w4a4_gemm", "w4a4_pair"],
                     help="time only this row (and the headline GEMV): for profiling runs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps

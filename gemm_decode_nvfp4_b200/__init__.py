@@ -197,6 +197,7 @@ def quantize_mse(w: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g_out: torch
 
 
 FLAG_STATIC_WEIGHTS = 1
+FLAG_W4A4_PAIR = 1 << 12
 
 
 def _ksplit_flag(k_split: int) -> int:
@@ -453,10 +454,11 @@ def _need_w4a4_weights(q: torch.Tensor, s_mma: torch.Tensor, g: torch.Tensor):
     return N, K
 
 
-def w4a4_gemm(qx, sx, x_amax, q, s_mma, g, Y, stream=None, static_weights: bool = False) -> None:
+def w4a4_gemm(qx, sx, x_amax, q, s_mma, g, Y, stream=None, static_weights: bool = False, pair: bool = False) -> None:
     """Y [M, N] = bf16(g * (x_amax[0] / 2688) * Xq . Wq^T) from quantized
     activations (qx, sx, x_amax from w4a4_quantize_x) and weights (q, s_mma
-    from w4a4_prepare_weights, g)."""
+    from w4a4_prepare_weights, g).  pair: tiles of 256 weight rows on pairs
+    of SMs (NVFP4_FLAG_W4A4_PAIR)."""
     _need(Y, torch.bfloat16, "Y", 2)
     _need(qx, torch.uint8, "qx", 2)
     _need(sx, torch.uint8, "sx")
@@ -467,7 +469,7 @@ def w4a4_gemm(qx, sx, x_amax, q, s_mma, g, Y, stream=None, static_weights: bool 
         raise ValueError(f"shape mismatch: qx {tuple(qx.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
     if sx.numel() < lib.nvfp4_w4a4_x_scales_bytes(M, K):
         raise ValueError(f"sx holds {sx.numel()} bytes, [{M}, {K}] needs {lib.nvfp4_w4a4_x_scales_bytes(M, K)}")
-    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    flags = (FLAG_STATIC_WEIGHTS if static_weights else 0) | (FLAG_W4A4_PAIR if pair else 0)
     dev = _device(qx, sx, x_amax, q, s_mma, g, Y)
     _call("nvfp4_w4a4_gemm", dev, _ptr(qx), _ptr(sx), _ptr(x_amax), _ptr(q), _ptr(s_mma), _ptr(g), _ptr(Y),
           Y.stride(0), M, N, K, flags, _stream(stream, dev))
@@ -479,7 +481,7 @@ def w4a4_workspace_size(M: int, K: int) -> int:
 
 def w4a4_linear(X: torch.Tensor, q: torch.Tensor, s_mma: torch.Tensor, g: torch.Tensor, Y: torch.Tensor,
                 workspace: torch.Tensor, x_amax: torch.Tensor | None = None, stream=None,
-                static_weights: bool = False) -> None:
+                static_weights: bool = False, pair: bool = False) -> None:
     """Y [M, N] = W4A4 product of BF16 X [M, K] (quantized on the fly into the
     workspace) and NVFP4 weights (q, s_mma from w4a4_prepare_weights, g)."""
     _need(X, torch.bfloat16, "X", 2)
@@ -491,7 +493,7 @@ def w4a4_linear(X: torch.Tensor, q: torch.Tensor, s_mma: torch.Tensor, g: torch.
     M, K = X.shape
     if Kq != K or Y.shape != (M, N):
         raise ValueError(f"shape mismatch: X {tuple(X.shape)}, q {tuple(q.shape)}, Y {tuple(Y.shape)}")
-    flags = FLAG_STATIC_WEIGHTS if static_weights else 0
+    flags = (FLAG_STATIC_WEIGHTS if static_weights else 0) | (FLAG_W4A4_PAIR if pair else 0)
     if X.stride(1) != 1:
         raise ValueError("X rows must be contiguous")
     dev = _device(X, x_amax, q, s_mma, g, Y, workspace)

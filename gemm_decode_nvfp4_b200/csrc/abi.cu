@@ -37,6 +37,7 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 constexpr uint32_t kKnownFlags = NVFP4_FLAG_STATIC_WEIGHTS;
 constexpr uint32_t kGemvFlags = NVFP4_FLAG_STATIC_WEIGHTS | NVFP4_FLAG_KSPLIT_MASK;
+constexpr uint32_t kW4a4Flags = NVFP4_FLAG_STATIC_WEIGHTS | NVFP4_FLAG_W4A4_PAIR;
 
 // The K split a decode GEMV call asks for (0 = the library's choice), or -1
 // for a value other than 1, 2, 4, 8.
@@ -486,7 +487,7 @@ nvfp4_status nvfp4_w4a4_quantize_x(const uint16_t* X, int64_t ldx, int64_t M, in
 nvfp4_status nvfp4_w4a4_gemm(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
                              const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
                              int64_t K, uint32_t flags, nvfp4_stream_t stream) {
-  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~kW4a4Flags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   nvfp4_status st = check_w4a4_shape(M, N, K);
   if (st != NVFP4_OK) return st;
   if (M == 0 || N == 0) return NVFP4_OK;
@@ -505,7 +506,8 @@ nvfp4_status nvfp4_w4a4_gemm(const uint8_t* qx, const uint8_t* sx, const float* 
   st = check_device(&sms);
   if (st != NVFP4_OK) return st;
   cudaError_t e = nvfp4::launch_gemm_w4a4(qx, sx, x_amax, q, s_mma, g, Y, ldy, M, N, K,
-                                          (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0, (cudaStream_t)stream, sms);
+                                          (flags & NVFP4_FLAG_STATIC_WEIGHTS) != 0, (flags & NVFP4_FLAG_W4A4_PAIR) != 0,
+                                          (cudaStream_t)stream, sms);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "W4A4 GEMM launch");
 }
 
@@ -513,7 +515,7 @@ nvfp4_status nvfp4_w4a4_linear(const uint16_t* X, int64_t ldx, const float* x_am
                                const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
                                int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
                                nvfp4_stream_t stream) {
-  if (flags & ~kKnownFlags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~kW4a4Flags) return fail(NVFP4_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   nvfp4_status st = check_w4a4_shape(M, N, K);
   if (st != NVFP4_OK) return st;
   if (M == 0 || N == 0) return NVFP4_OK;

@@ -328,6 +328,282 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------ pair-of-SMs tile
+//
+// The same GEMM on tiles of 256 weight rows x 256 tokens run by a cluster of
+// two CTAs on two SMs (tcgen05 cta_group::2): each CTA holds its 128 weight
+// rows (the pair's MMA has M = 256) and half of the tile's tokens (B rows
+// 128 r .. 128 r + 127 of CTA rank r), so a token tile crosses from L2 into
+// the SMs once per 256 weight rows instead of once per 128.  The even CTA
+// issues the scale copies and the MMAs for both; each CTA's tensor memory
+// holds its 128 accumulator rows x 256 tokens and the scale factors of its
+// own weight rows and of all 256 tokens (each CTA loads the token scales in
+// full).  A stage is 38 KB (16 KB of weight codes, 16 KB of token codes,
+// 2 + 4 KB of scale atoms), so five stages fit beside the epilogue.
+//   - warp 0 of each CTA: TMA of its own stage bytes (codes and scale atoms)
+//     into its own shared memory, all counted on the even CTA's `full`
+//     (the odd CTA's loads use the pair form of the tensor copy);
+//   - warp 1 of the even CTA: the MMA issuer; its commits arrive on both
+//     CTAs' barriers;
+//   - warps 2..5: the epilogue of each CTA's accumulator rows; the even
+//     CTA's issuer waits for both epilogues (acc_empty, 8 arrivals) before it
+//     overwrites the accumulator.
+constexpr int kPairStages = 5;
+constexpr int kPairBBytes = (kBN / 2) * 128;          // this CTA's 128 tokens of a stage
+constexpr int kPairStageBytes = kABytes + kPairBBytes + kSFABytes + kSFBBytes;
+constexpr uint32_t kPairIdesc = ptx::idesc_nvf4(2 * kBM, kBN);
+static_assert(kPairStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle)");
+static_assert(kSfCol0 + kPairStages * 4 * kSfColsPerMma <= kTmemCols, "TMEM columns");
+
+struct PairBars {
+  uint64_t full[kPairStages];       // (even CTA) both CTAs' bytes of the stage have landed
+  uint64_t empty[kPairStages];      // the pair's MMAs that read the stage are done
+  uint64_t acc_full;                // the tile's accumulator is complete
+  uint64_t acc_empty;               // (even CTA) both CTAs' epilogues have read it
+  uint64_t mma_done;                // every MMA of the pair has finished (teardown)
+  uint32_t tmem_addr;
+  volatile int err;
+};
+
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + kEpiBytes + (int)sizeof(PairBars) + 1024;
+static_assert(kPairSmemBytes <= 232448, "shared memory per CTA");
+
+__device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairBars* bars) {
+  if (bars->err) return false;
+  if (ptx::mbar_wait_cluster(bar, parity, kWaitLimitNs)) return true;
+  if (!bars->err) {
+    bars->err = 1;
+    atomicAdd(&g_w4a4_wait_timeouts, 1u);
+  }
+  return false;
+}
+
+// Persistent pairs: cluster c = blockIdx.x / 2 takes the pair tiles
+// t = c, c + gridDim.x / 2, ... (weight rows 256 (t % tiles_n), tokens
+// 256 (t / tiles_n)); both CTAs walk the same tiles and stages.
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                          const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
+                          const float* __restrict__ g, const float* __restrict__ x_amax, uint16_t* __restrict__ Y,
+                          int64_t ldy, int M, int N, int K, int static_weights) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = ptx::smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  auto a_tile = [&](int st) { return smem + st * kPairStageBytes; };
+  auto b_tile = [&](int st) { return smem + st * kPairStageBytes + kABytes; };
+  auto sfa = [&](int st) { return smem + st * kPairStageBytes + kABytes + kPairBBytes; };
+  auto sfb = [&](int st) { return smem + st * kPairStageBytes + kABytes + kPairBBytes + kSFABytes; };
+  uint8_t* epi = smem + kPairStages * kPairStageBytes;
+  PairBars* bars = reinterpret_cast<PairBars*>(epi + kEpiBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the pair's MMAs
+  const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+  const int steps64 = K / 64;
+  const int num_ks = K / kStageK;
+  const int tiles_n = (N + 2 * kBM - 1) / (2 * kBM);
+  const int tiles = tiles_n * ((M + kBN - 1) / kBN);
+  const int scale_tiles = (N + kBM - 1) / kBM;  // 128-row tiles of s_mma
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kPairStages; ++st) {
+      ptx::mbar_init(&bars->full[st], 1);
+      ptx::mbar_init(&bars->empty[st], 1);
+    }
+    ptx::mbar_init(&bars->acc_full, 1);
+    ptx::mbar_init(&bars->acc_empty, 2 * kEpiWarps);
+    ptx::mbar_init(&bars->mma_done, 1);
+    bars->err = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmap_w);
+    ptx::prefetch_tmap(&tmap_x);
+    ptx::prefetch_tmap(&tmap_sa);
+    ptx::prefetch_tmap(&tmap_sb);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(&bars->tmem_addr, kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before either signals the other
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_addr;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int gi = 0;  // stages issued so far (over all tiles of this pair)
+      bool first = true;
+      for (int t = cluster; t < tiles && !bars->err; t += clusters) {
+        const int nt = t % tiles_n, mt = t / tiles_n;
+        const int n0 = nt * 2 * kBM + (int)rank * kBM, m0 = mt * kBN;
+        // the odd CTA's rows may lie past N: its scale atoms then come from
+        // the last tile (its codes read as zero; its outputs are not stored)
+        const int sa_tile = n0 / kBM < scale_tiles ? n0 / kBM : scale_tiles - 1;
+        // scale maps: rows of 256 bytes, a stage's four 512-byte atoms are 8 rows
+        const int sa_row = sa_tile * steps64 * 2, sb_row0 = 2 * mt * steps64 * 2, sb_row1 = (2 * mt + 1) * steps64 * 2;
+        auto issue = [&](int st, int ks, bool weights, bool tokens) {
+          if (rank == 0) {
+            if (weights) {
+              ptx::tma_load_2d(a_tile(st), &tmap_w, &bars->full[st], ks * 128, n0);
+              ptx::tma_load_2d(sfa(st), &tmap_sa, &bars->full[st], 0, sa_row + ks * 8);
+            }
+            if (tokens) {
+              ptx::tma_load_2d(b_tile(st), &tmap_x, &bars->full[st], ks * 128, m0);
+              ptx::tma_load_2d(sfb(st), &tmap_sb, &bars->full[st], 0, sb_row0 + ks * 8);
+              ptx::tma_load_2d(sfb(st) + 2048, &tmap_sb, &bars->full[st], 0, sb_row1 + ks * 8);
+            }
+          } else {
+            const uint32_t fb = ptx::cluster_addr(&bars->full[st], 0);
+            if (weights) {
+              ptx::tma_load_2d_pair(a_tile(st), &tmap_w, fb, ks * 128, n0);
+              ptx::tma_load_2d_pair(sfa(st), &tmap_sa, fb, 0, sa_row + ks * 8);
+            }
+            if (tokens) {
+              ptx::tma_load_2d_pair(b_tile(st), &tmap_x, fb, ks * 128, m0 + kBN / 2);
+              ptx::tma_load_2d_pair(sfb(st), &tmap_sb, fb, 0, sb_row0 + ks * 8);
+              ptx::tma_load_2d_pair(sfb(st) + 2048, &tmap_sb, fb, 0, sb_row1 + ks * 8);
+            }
+          }
+        };
+        int ks = 0;
+        if (first) {
+          const int f = num_ks < kPairStages ? num_ks : kPairStages;
+          // the even CTA's barrier counts both CTAs' bytes of each stage
+          if (rank == 0)
+            for (int k = 0; k < f; ++k) ptx::mbar_arrive_expect_tx(&bars->full[k], 2 * kPairStageBytes);
+          if (static_weights)
+            for (int k = 0; k < f; ++k) issue(k, k, true, false);
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          for (int k = 0; k < f; ++k) issue(k, k, !static_weights, true);
+          ks = f;
+          gi = f;
+          first = false;
+        }
+        for (; ks < num_ks; ++ks) {
+          const int st = gi % kPairStages;
+          if (gi >= kPairStages && !pair_wait(&bars->empty[st], ((gi / kPairStages) - 1) & 1, bars)) break;
+          if (rank == 0) ptx::mbar_arrive_expect_tx(&bars->full[st], 2 * kPairStageBytes);
+          issue(st, ks, true, true);
+          ++gi;
+        }
+      }
+      if (bars->err && rank == 0) {
+        // let copies already issued land before the CTA exits (the odd CTA's
+        // land on the even CTA's barriers, which this waits for too)
+        for (int j = gi > kPairStages ? gi - kPairStages : 0; j < gi; ++j)
+          ptx::mbar_wait_cluster(&bars->full[j % kPairStages], (j / kPairStages) & 1, kWaitLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (rank == 0) {
+        // ------------------------------------------- MMA issuer for the pair
+        int gi = 0, it = 0;
+        for (int t = cluster; t < tiles; t += clusters, ++it) {
+          // the accumulator is free once both epilogues have read the previous tile
+          if (it > 0) {
+            if (!pair_wait(&bars->acc_empty, (it - 1) & 1, bars)) break;
+            ptx::tc_fence_after();
+          }
+          bool ok = true;
+          for (int ks = 0; ks < num_ks; ++ks, ++gi) {
+            const int st = gi % kPairStages;
+            const uint32_t par = (uint32_t)(gi / kPairStages) & 1u;
+            if (!pair_wait(&bars->full[st], par, bars)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t a0 = ptx::smem_u32(a_tile(st)), b0 = ptx::smem_u32(b_tile(st));
+            const uint32_t fa = ptx::smem_u32(sfa(st)), fb = ptx::smem_u32(sfb(st));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma;
+              ptx::tmem_copy_sf_pair(col, ptx::rows16_desc(fa + kk * 512));
+              ptx::tmem_copy_sf_pair(col + 4, ptx::rows16_desc(fb + kk * 512));
+              ptx::tmem_copy_sf_pair(col + 8, ptx::rows16_desc(fb + 2048 + kk * 512));
+              ptx::mma_nvf4_pair(tmem, ptx::sw128_kmajor_desc(a0 + 32 * kk), ptx::sw128_kmajor_desc(b0 + 32 * kk),
+                                 kPairIdesc, col, col + 4, (ks | kk) != 0);
+            }
+            ptx::mma_commit_pair(&bars->empty[st]);
+          }
+          if (!ok) break;
+          ptx::mma_commit_pair(&bars->acc_full);
+        }
+        // arrives in both CTAs when every MMA above is done (also on the
+        // error path), so that neither frees its tensor memory under an MMA
+        ptx::mma_commit_pair(&bars->mma_done);
+      }
+      ptx::mbar_wait_cluster(&bars->mma_done, 0, kWaitLimitNs);
+    }
+  } else {
+    // ----------------------------------------------------------------- epilogue
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // x_amax and Y
+    const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. +31 = this CTA's weight rows
+    const float scale = __fmul_rn(*g, __fdiv_rn(*x_amax, 2688.0f));
+    const uint32_t stage = ptx::smem_u32(epi) + (uint32_t)(warp - kEpiWarp0) * 2048u;
+    const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+    int it = 0;
+    for (int t = cluster; t < tiles; t += clusters, ++it) {
+      const int nt = t % tiles_n, mt = t / tiles_n;
+      const int n0 = nt * 2 * kBM + (int)rank * kBM, m0 = mt * kBN;
+      if (!__all_sync(0xFFFFFFFFu, pair_wait(&bars->acc_full, it & 1, bars))) break;
+      ptx::tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBN && m0 + c0 < M; c0 += 32) {
+        uint32_t rr[32];
+        ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(rr[j]) * scale);
+          st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
+          const int m = m0 + c0 + j;
+          const int nb = n0 + 32 * quarter + 8 * piece;
+          if (m < M && nb < N) {
+            const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
+            uint16_t* dst = Y + (int64_t)m * ldy + nb;
+            if (vec_ok && nb + 8 <= N) {
+              *reinterpret_cast<uint4*>(dst) = v;
+            } else {
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+              for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
+            }
+          }
+        }
+        __syncwarp();
+      }
+      // every TMEM read of this tile has completed (tcgen05.wait::ld above)
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          ptx::mbar_arrive(&bars->acc_empty);
+        else
+          ptx::mbar_arrive_remote(&bars->acc_empty, 0);
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // neither CTA leaves while the other may still signal it or read its shared memory
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
 // ------------------------------------------------- activations for W4A4 GEMMs
 //
 // X [M, K] quantized by the weights' rule with g_x = x_amax / 2688: codes
@@ -459,17 +735,52 @@ cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t
 
 cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
                              const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
-                             int64_t K, bool static_weights, cudaStream_t stream, int sms) {
+                             int64_t K, bool static_weights, bool pair, cudaStream_t stream, int sms) {
   CUtensorMap tw, tx;
   if (!tc::make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2),
                         128u, (uint32_t)kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !tc::make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, (uint64_t)(K / 2), (uint64_t)M, (uint64_t)(K / 2),
                         128u, (uint32_t)kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  int m = (int)M, n = (int)N, k = (int)K, sw = static_weights ? 1 : 0;
+  if (pair && sms >= 2) {
+    // pairs of SMs: the token map's box is the 128 tokens one CTA of a pair loads
+    // and the scale atoms as rows of 256 bytes (a stage's four atoms: 8 rows)
+    CUtensorMap txh, tsa, tsb;
+    const uint64_t sa_rows = (uint64_t)((N + kBM - 1) / kBM) * (uint64_t)(K / 64) * 2;
+    const uint64_t sb_rows = (uint64_t)((M + kBN - 1) / kBN * 2) * (uint64_t)(K / 64) * 2;
+    if (!tc::make_tmap_2d(&txh, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, (uint64_t)(K / 2), (uint64_t)M, (uint64_t)(K / 2),
+                          128u, (uint32_t)(kBN / 2), CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !tc::make_tmap_2d(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT8, s_mma, 256u, sa_rows, 256u, 256u, 8u,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !tc::make_tmap_2d(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, sx, 256u, sb_rows, 256u, 256u, 8u,
+                          CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    static tc::SmemOptIn opt_in_pair;
+    const cudaError_t e = opt_in_pair.ensure((const void*)gemm_w4a4_pair_kernel, kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    void* args[] = {&tw, &txh, &tsa, &tsb, (void*)&g, (void*)&x_amax, &Y, &ldy, &m, &n, &k, &sw};
+    const int64_t tiles = (N + 2 * kBM - 1) / (2 * kBM) * ((M + kBN - 1) / kBN);
+    const int64_t clusters = tiles < sms / 2 ? tiles : sms / 2;  // one persistent pair per two SMs at most
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelExC(&cfg, (const void*)gemm_w4a4_pair_kernel, args);
+  }
   static tc::SmemOptIn opt_in;
   const cudaError_t e = opt_in.ensure((const void*)gemm_w4a4_kernel, kSmemBytes);
   if (e != cudaSuccess) return e;
-  int m = (int)M, n = (int)N, k = (int)K, sw = static_weights ? 1 : 0;
   void* args[] = {&tw, &tx, (void*)&s_mma, (void*)&sx, (void*)&g, (void*)&x_amax, &Y, &ldy, &m, &n, &k, &sw};
   const int64_t tiles = (N + kBM - 1) / kBM * ((M + kBN - 1) / kBN);
   const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);  // one persistent CTA per SM at most

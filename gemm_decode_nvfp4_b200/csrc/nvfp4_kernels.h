@@ -59,7 +59,7 @@ cudaError_t launch_scales_to_mma(const uint8_t* s, int64_t N, int64_t K, uint8_t
                                  int sms);
 cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
                              const uint8_t* s_mma, const float* g, uint16_t* Y, int64_t ldy, int64_t M, int64_t N,
-                             int64_t K, bool static_weights, cudaStream_t stream, int sms);
+                             int64_t K, bool static_weights, bool pair, cudaStream_t stream, int sms);
 cudaError_t read_and_clear_w4a4_timeouts(unsigned int* count);
 // MXFP4 scales restated as NVFP4 scales s_nv [N, K/16] and a power-of-two
 // tensor scale g (quantize.cu); non-zero blocks outside the E4M3 window are

@@ -98,6 +98,19 @@ typedef enum nvfp4_status {
 #define NVFP4_FLAG_KSPLIT(c) (((uint32_t)(c) & 15u) << 8)
 #define NVFP4_FLAG_KSPLIT_MASK (15u << 8)
 
+/*
+ * W4A4 GEMM only (nvfp4_w4a4_gemm, nvfp4_w4a4_linear): NVFP4_FLAG_W4A4_PAIR
+ * runs the GEMM on tiles of 256 weight rows x 256 tokens, each on a pair of
+ * SMs (a 2-CTA cluster whose even CTA issues tcgen05.mma.cta_group::2 for
+ * both): a token tile then crosses from L2 into the SMs once per 256 weight
+ * rows instead of once per 128.  The result is the same as without the flag
+ * (same products, same fp32 accumulation order per output).  On one B200 the
+ * [17408, 5120] layer at M = 512 ran at 38.7 us per call with the flag and
+ * 35.3 us without (each stage then waits for the later of two CTAs' loads),
+ * so it is off by default.
+ */
+#define NVFP4_FLAG_W4A4_PAIR (1u << 12)
+
 /* Version of this ABI (major * 10000 + minor * 100 + patch). */
 NVFP4_API int nvfp4_version(void);
 

@@ -77,7 +77,8 @@ NVFP4_API nvfp4_status nvfp4_w4a4_quantize_x(const uint16_t* X, int64_t ldx, int
 /*
  * Y = bf16(g * (x_amax / 2688) * Xq . Wq^T) from quantized activations (qx,
  * sx, x_amax as nvfp4_w4a4_quantize_x leaves them) and weights (q, s_mma from
- * nvfp4_w4a4_prepare_weights, g).  flags: NVFP4_FLAG_STATIC_WEIGHTS (nvfp4.h).
+ * nvfp4_w4a4_prepare_weights, g).  flags: NVFP4_FLAG_STATIC_WEIGHTS and
+ * NVFP4_FLAG_W4A4_PAIR (nvfp4.h).
  * Y must not overlap any input.  M == 0 or N == 0 is a no-op.
  */
 NVFP4_API nvfp4_status nvfp4_w4a4_gemm(const uint8_t* qx, const uint8_t* sx, const float* x_amax, const uint8_t* q,
@@ -90,7 +91,7 @@ NVFP4_API size_t nvfp4_w4a4_workspace_size(int64_t M, int64_t K);
 /*
  * nvfp4_w4a4_quantize_x into the workspace, then nvfp4_w4a4_gemm.  x_amax:
  * NULL for the dynamic max |X|, else a device pointer to a calibrated amax.
- * flags: NVFP4_FLAG_STATIC_WEIGHTS.  The workspace (at least
+ * flags: NVFP4_FLAG_STATIC_WEIGHTS, NVFP4_FLAG_W4A4_PAIR.  The workspace (at least
  * nvfp4_w4a4_workspace_size(M, K) bytes) must not overlap the other buffers;
  * calls that share it must be ordered on one stream.
  */

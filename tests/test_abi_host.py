@@ -205,3 +205,15 @@ def test_mxfp4_to_nvfp4_scales_validation():
     assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 8192, A + 12290, None) == ALIGN   # g_out
     assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 64, A + 12288, None) == INVALID   # s_nv in q
     assert L.mxfp4_to_nvfp4_scales(A, A + 4096, 4, 64, A + 8192, A + 4100, None) == INVALID  # g_out in s_mx
+
+
+def test_w4a4_pair_flag():
+    """NVFP4_FLAG_W4A4_PAIR (bit 12) is taken by the W4A4 entry points only;
+    the flags are checked before any device work (M == 0 is a no-op)."""
+    pair = nv.FLAG_W4A4_PAIR
+    assert pair == 1 << 12
+    assert nv.lib.nvfp4_w4a4_gemm(A, A, A, A, A, A, A + 4096, 64, 0, 64, 256, pair | 1, None) == OK
+    assert nv.lib.nvfp4_w4a4_gemm(A, A, A, A, A, A, A + 4096, 64, 0, 64, 256, 1 << 13, None) == INVALID
+    assert nv.lib.nvfp4_w4a4_linear(A, 256, None, A, A, A, A + 4096, 64, 0, 64, 256, A + 8192, 0, pair, None) == OK
+    assert nv.lib.nvfp4_gemm_ex(A, 64, A, A, A, A + 4096, 64, 4, 64, 64, None, 0, pair, None) == INVALID
+    assert nv.lib.nvfp4_gemv_ex(A, A, A, A, A + 4096, 4, 1024, pair, None) == INVALID

@@ -87,7 +87,7 @@ def test_quantize_x_given_amax_and_strided_rows(nv):
     assert np.array_equal(from_mma_layout(sx.cpu().numpy(), 96, 1024, 256)[:96], s_ref)
 
 
-def _run(nv, X, q, s, g, x_amax=None, static=False):
+def _run(nv, X, q, s, g, x_amax=None, static=False, pair=False):
     M, K = X.shape
     N = q.shape[0]
     qd, sd = torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda()
@@ -96,33 +96,47 @@ def _run(nv, X, q, s, g, x_amax=None, static=False):
     ws = torch.empty((nv.w4a4_workspace_size(M, K),), dtype=torch.uint8, device="cuda")
     Y, check = guarded_empty((M, N), torch.bfloat16)
     am = None if x_amax is None else torch.tensor([x_amax], dtype=torch.float32, device="cuda")
-    nv.w4a4_linear(X.cuda(), qd, s_mma, gd, Y, ws, x_amax=am, static_weights=static)
+    nv.w4a4_linear(X.cuda(), qd, s_mma, gd, Y, ws, x_amax=am, static_weights=static, pair=pair)
     check()
     nv.check_device_errors()
     return Y
 
 
+@pytest.mark.parametrize("pair", [False, True], ids=["sm", "pair"])
 @pytest.mark.parametrize("M,N,K", [(256, 256, 1024),   # one tile, four stages
                                    (300, 1000, 2048),  # ragged M and N tiles, a ring wrap
                                    (1, 130, 256),      # one token, one stage
                                    (40, 384, 1280),    # five stages on a four-stage ring
+                                   (40, 1100, 1536),   # pairs: the last pair's odd CTA is past N
                                    (513, 128, 512)])   # three token tiles
-def test_w4a4_gemm_vs_oracle(nv, M, N, K):
+def test_w4a4_gemm_vs_oracle(nv, M, N, K, pair):
     X = workloads.activations(M, K, 7 * M + K)
     q, s, g = oracle.quantize(workloads.random_bf16((N, K), N + K))
-    Y = _run(nv, X, q, s, g)
+    Y = _run(nv, X, q, s, g, pair=pair)
     y_ref, bound, _ = oracle.w4a4_linear(X, q, s, g)
-    assert_within_tolerance(Y, y_ref, bound, f"w4a4 M={M} N={N} K={K}")
+    assert_within_tolerance(Y, y_ref, bound, f"w4a4 M={M} N={N} K={K} pair={pair}")
 
 
-def test_w4a4_full_size_sampled(nv):
+@pytest.mark.parametrize("M,N,K", [(300, 1100, 2048), (512, 2048, 5120)])
+def test_w4a4_pair_tiles_equal_single(nv, M, N, K):
+    """Tiles on pairs of SMs form the same products and fp32 sums per output
+    as tiles on one SM: the outputs agree bit for bit."""
+    X = workloads.activations(M, K, M + 3 * K)
+    q, s, g = oracle.quantize(workloads.random_bf16((N, K), N + 5))
+    Y1 = _run(nv, X, q, s, g, pair=False)
+    Y2 = _run(nv, X, q, s, g, pair=True)
+    assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("pair", [False, True], ids=["sm", "pair"])
+def test_w4a4_full_size_sampled(nv, pair):
     """The 27B-class prefill layer: M = 512 tokens, W [17408, 5120]."""
     cfg = workloads.CONFIGS["prefill"]
     M, N, K = cfg.M, cfg.N, cfg.K
     w = workloads.weight_bf16(cfg)
     q, s, g = oracle.quantize(w)
     X = workloads.activations(M, K, cfg.seed + 1)
-    Y = _run(nv, X, q, s, g, static=True)
+    Y = _run(nv, X, q, s, g, static=True, pair=pair)
     rng = np.random.default_rng(5)
     rows, cols = rng.integers(0, M, 600), rng.integers(0, N, 600)
     y_ref, bound, _ = oracle.w4a4_linear(X, q, s, g, rows=rows, cols=cols)
