@@ -53,9 +53,10 @@ namespace {
 constexpr int kBM = 128;        // weight rows per CTA (MMA M)
 constexpr int kBK = 64;         // k per A tile (one 128-byte row of f16)
 constexpr int kWK = 256;        // k per weight stage (one 128-byte line of codes per row)
-// Warp roles: producer, four MMA issuers (an MMA instruction costs its issuing
-// warp about 45 cycles at these N whatever the tile, so one issuer per
-// dequantization group keeps the tensor cores fed), converter, 16 dequantizers.
+// Warp roles: producer, four MMA issuers (a lone thread issues one MMA about
+// every 56 cycles at these N, while the tensor pipe needs 16 for an N = 32
+// MMA, so one issuer per dequantization group keeps it supplied), converter,
+// 16 dequantizers.
 constexpr int kProdWarp = 0, kMmaWarp0 = 1, kMmaWarps = 4, kConvWarp = 5, kDeqWarp0 = 6, kDeqWarps = 16;
 // M > 8: one f16-activation producer warp per MMA issuer, so that each
 // issuer's activation tiles are refilled as soon as its own MMAs release them
@@ -342,8 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!CONV) {
           // one wait for the B tile and one for the half stage's second A
           // sub-slot: the same 128 threads signal the first sub-slot before
-          // the second, so its phase is complete too (each wait costs this
-          // warp hundreds of cycles, whether or not the phase is complete)
+          // the second, so its phase is complete too (fewer waits: with the
+          // dequantization warps storing into tensor memory, this warp's
+          // waits and MMAs take several times their cost in an idle CTA)
           if (!wait_or_fail(&bars->xfull[xs], (h / NX) & 1, bars)) break;
           const int s1 = sidx + 1;
           if (!wait_or_fail(&bars->afull[gi * C::kNS + s1 % C::kNS], (s1 / C::kNS) & 1, bars)) break;
