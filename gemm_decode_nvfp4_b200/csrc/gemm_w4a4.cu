@@ -24,15 +24,26 @@
 //   - warp 0, one thread: TMA loads of the weight codes [128, 128 B] and the
 //     token codes [256, 128 B] (out-of-range rows read as zero) and bulk
 //     copies of the stage's scale atoms (2 KB of weights, 2 x 2 KB of tokens);
-//   - warp 1, one thread: per MMA, three tcgen05.cp of its scale atoms into
-//     the stage's own TMEM columns, then the MMA into the [128 x 256] fp32
-//     accumulator; each stage is committed to its "empty" barrier;
-//   - warps 2..5: the epilogue, TMEM -> g * g_x -> BF16 Y through shared memory.
+//   - warps 18..20, one thread each: warp 18 + j copies atom j of every MMA
+//     (j = 0: weight scales, 1 and 2: the two halves of the token scales)
+//     into the stage's own TMEM columns with tcgen05.cp, committed per stage
+//     to "sf_full" (three arrivals);
+//   - warp 1, one thread: the four MMAs of a stage into the [128 x 256] fp32
+//     accumulator once its codes ("full") and scale factors ("sf_full") are
+//     in; each stage is committed to its "empty" barrier;
+//   - warps 2..17: the epilogue, TMEM -> g * g_x -> BF16 Y, four warps per
+//     TMEM lane quarter, each with two of the tile's eight 32-column blocks.
+// The copies have threads of their own because one thread issues a tcgen05
+// instruction only every few tens of cycles: with the twelve copies and four
+// MMAs of a stage in one thread, the issue took longer than the tensor pipe's
+// work (35.0 µs on the 512 x 17408 x 5120 layer, 26.5 µs with the copies
+// left out, 32.2 µs with them in one thread of their own).
 // The kernel is persistent (one CTA per SM, tiles in a fixed stride), so
 // the next tile's stages stream in while the epilogue drains the accumulator.
 // A stage's TMEM scale columns are rewritten only after the MMAs that read
-// them have completed (the stage's empty barrier), and tcgen05.cp is ordered
-// before the MMAs its thread issues after it.  Every wait is bounded.
+// them have completed: the copy warp rewrites them after the stage's next
+// "full", which follows its "empty" (the MMAs' commit) and the reload.
+// Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -59,8 +70,11 @@ constexpr int kBBytes = kBN * 128;            // packed token codes of a stage
 constexpr int kSFABytes = 4 * 512;            // weight scale atoms (4 MMAs)
 constexpr int kSFBBytes = 2 * 4 * 512;        // token scale atoms (2 x 128 tokens, 4 MMAs)
 constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-constexpr int kThreads = 6 * 32;
-constexpr int kEpiWarp0 = 2;
+constexpr int kEpiWarp0 = 2, kEpiWarps = 16;  // epilogue: four warps per TMEM lane quarter
+static_assert(kEpiWarps % 4 == 0, "every TMEM lane quarter has the same number of epilogue warps");
+constexpr int kEpiBytes = kEpiWarps * 512;     // each epilogue warp's 8 tokens x 32 rows BF16 staging block
+constexpr int kSfWarp0 = kEpiWarp0 + kEpiWarps, kSfWarps = 3;  // scale-factor copies, one warp per atom
+constexpr int kThreads = (kSfWarp0 + kSfWarps) * 32;
 constexpr uint32_t kTmemCols = 512;           // 256 accumulator + 4 stages x 4 MMAs x 12 scale columns
 constexpr uint32_t kSfCol0 = 256;
 constexpr uint32_t kSfColsPerMma = 12;        // 4 weight + 8 token columns
@@ -69,12 +83,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle)");
 static_assert(kSfCol0 + kStages * 4 * kSfColsPerMma <= kTmemCols, "TMEM columns");
 
-constexpr int kEpiWarps = 4;
-constexpr int kEpiBytes = kEpiWarps * 2048;  // each epilogue warp's 32 x 32 BF16 staging block
-
 struct Bars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t sf_full[kStages];  // the stage's scale factors are in tensor memory (the copy warps' commits)
+  uint64_t sf_done;           // every scale-factor copy of the CTA has finished (teardown)
   uint64_t acc_full;   // the accumulator of the current tile is complete (one phase per tile)
   uint64_t acc_empty;  // the epilogue has read it (kEpiWarps arrivals per tile)
   uint64_t mma_done;   // every MMA of the CTA has finished (teardown)
@@ -95,6 +108,28 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Bar
   return false;
 }
 
+// A wait that spans a whole main loop (the epilogue's): the thread sleeps
+// between polls instead of taking issue slots from the producer, copy and MMA
+// threads.  Bounded like every other wait.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait_sleep(bar, parity))
+    if (ptx::globaltimer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
+// wait_or_fail with the sleeping wait
+__device__ __forceinline__ bool wait_or_fail_sleep(uint64_t* bar, uint32_t parity, Bars* bars) {
+  if (bars->err) return false;
+  if (mbar_wait_sleep(bar, parity, kWaitLimitNs)) return true;
+  if (!bars->err) {
+    bars->err = 1;
+    atomicAdd(&g_w4a4_wait_timeouts, 1u);
+  }
+  return false;
+}
+
 __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
   asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
@@ -104,6 +139,48 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
                : "memory");
   return v;
+}
+
+// Epilogue of a [128 weight rows x 256 tokens] fp32 accumulator tile: the
+// warp reads the TMEM lane quarter its index fixes (warp % 4: a warp may only
+// reach those 32 lanes, its weight rows) and the 32-column blocks p, p + 4
+// (tokens) for its rank p = (warp - kEpiWarp0) / 4 among the epilogue warps
+// of that quarter, scales by `scale` and stores BF16 Y[m, n], eight tokens
+// at a time through its 512 bytes of shared memory at `stage` so that each
+// lane stores 16 bytes (a quarter of a token's 32 rows).
+__device__ __forceinline__ void store_tile(uint32_t tmem, int warp, int lane, float scale, uint32_t stage,
+                                           uint16_t* __restrict__ Y, int64_t ldy, int M, int N, int m0, int n0) {
+  const int quarter = warp & 3, part = (warp - kEpiWarp0) >> 2;
+  const int jj = lane >> 2, piece = lane & 3;  // this lane's 16 bytes of a round: token jj, rows 8 piece ..
+  const int nb = n0 + 32 * quarter + 8 * piece;
+  const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+#pragma unroll 1
+  for (int c0 = 32 * part; c0 < kBN && m0 + c0 < M; c0 += 32 * (kEpiWarps / 4)) {
+    uint32_t rr[32];
+    ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {  // tokens c0 + 8 r .. c0 + 8 r + 7
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(rr[8 * r + j]) * scale);
+        st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
+      }
+      __syncwarp();
+      const int m = m0 + c0 + 8 * r + jj;
+      if (m < M && nb < N) {
+        const uint4 v = ld_shared_v4(stage + (uint32_t)(jj * 32 + 8 * piece) * 2u);
+        uint16_t* dst = Y + (int64_t)m * ldy + nb;
+        if (vec_ok && nb + 8 <= N) {
+          *reinterpret_cast<uint4*>(dst) = v;
+        } else {
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
+        }
+      }
+      __syncwarp();
+    }
+  }
 }
 
 // Rows of the weight scale rearrangement: thread t writes the 16 bytes of
@@ -157,7 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int st = 0; st < kStages; ++st) {
       ptx::mbar_init(&bars->full[st], 1);
       ptx::mbar_init(&bars->empty[st], 1);
+      ptx::mbar_init(&bars->sf_full[st], kSfWarps);
     }
+    ptx::mbar_init(&bars->sf_done, kSfWarps);
     ptx::mbar_init(&bars->acc_full, 1);
     ptx::mbar_init(&bars->acc_empty, kEpiWarps);
     ptx::mbar_init(&bars->mma_done, 1);
@@ -243,19 +322,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int ks = 0; ks < num_ks; ++ks, ++gi) {
           const int st = gi % kStages;
-          if (!wait_or_fail(&bars->full[st], (gi / kStages) & 1, bars)) {
+          // the stage's codes (TMA) and its scale factors (the copy warp)
+          if (!wait_or_fail(&bars->full[st], (gi / kStages) & 1, bars) ||
+              !wait_or_fail(&bars->sf_full[st], (gi / kStages) & 1, bars)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t a0 = ptx::smem_u32(a_tile(st)), b0 = ptx::smem_u32(b_tile(st));
-          const uint32_t fa = ptx::smem_u32(sfa(st)), fb = ptx::smem_u32(sfb(st));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma;
-            ptx::tmem_copy_sf(col, ptx::rows16_desc(fa + kk * 512));
-            ptx::tmem_copy_sf(col + 4, ptx::rows16_desc(fb + kk * 512));
-            ptx::tmem_copy_sf(col + 8, ptx::rows16_desc(fb + 2048 + kk * 512));
             ptx::mma_nvf4(tmem, ptx::sw128_kmajor_desc(a0 + 32 * kk), ptx::sw128_kmajor_desc(b0 + 32 * kk),
                           kIdesc, col, col + 4, (ks | kk) != 0);
           }
@@ -269,50 +346,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mma_commit(&bars->mma_done);
       ptx::mbar_wait(&bars->mma_done, 0, kWaitLimitNs);
     }
+  } else if (warp >= kSfWarp0) {
+    // ------------------------------------------- scale factors into tensor memory
+    // copy warp j: atom j of each MMA (weights, tokens 0-127, tokens 128-255),
+    // four 512-byte copies per stage, ahead of the MMAs (a slot's columns are
+    // rewritten only after its next `full`: after the MMAs that read them)
+    const uint32_t j = (uint32_t)(warp - kSfWarp0);
+    if (lane == 0) {
+      int gi = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        for (int ks = 0; ks < num_ks; ++ks, ++gi) {
+          const int st = gi % kStages;
+          if (!wait_or_fail(&bars->full[st], (gi / kStages) & 1, bars)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          // atom j of MMA kk: weights at sfa + 512 kk, tokens at sfb + 2048 (j - 1) + 512 kk
+          const uint32_t src = j == 0 ? ptx::smem_u32(sfa(st)) : ptx::smem_u32(sfb(st)) + 2048u * (j - 1);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma + 4u * j;
+            ptx::tmem_copy_sf(col, ptx::rows16_desc(src + kk * 512));
+          }
+          ptx::mma_commit(&bars->sf_full[st]);
+        }
+      }
+      // arrives when every copy above is done, so that TMEM is never freed
+      // under a running copy (also on the error path)
+      ptx::mma_commit(&bars->sf_done);
+      ptx::mbar_wait(&bars->sf_done, 0, kWaitLimitNs);
+    }
   } else {
     // ----------------------------------------------------------------- epilogue
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x_amax and Y
-    const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. +31 = weight rows of the tile
     const float scale = __fmul_rn(*g, __fdiv_rn(*x_amax, 2688.0f));
-    // each 32 x 32 block (weight rows of this quarter x tokens) goes through
-    // this warp's 2 KB so that Y is written as 64-byte runs
-    const uint32_t stage = ptx::smem_u32(epi) + (uint32_t)(warp - kEpiWarp0) * 2048u;
-    const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+    const uint32_t stage = ptx::smem_u32(epi) + (uint32_t)(warp - kEpiWarp0) * 512u;
     int it = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
       const int nt = t % tiles_n, mt = t / tiles_n;
-      const int n0 = nt * kBM, m0 = mt * kBN;
-      if (!__all_sync(0xFFFFFFFFu, wait_or_fail(&bars->acc_full, it & 1, bars))) break;
+      if (!__all_sync(0xFFFFFFFFu, wait_or_fail_sleep(&bars->acc_full, it & 1, bars))) break;
       ptx::tc_fence_after();
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBN && m0 + c0 < M; c0 += 32) {
-        uint32_t rr[32];
-        ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(rr[j]) * scale);
-          st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
-        }
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
-          const int m = m0 + c0 + j;
-          const int nb = n0 + 32 * quarter + 8 * piece;
-          if (m < M && nb < N) {
-            const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
-            uint16_t* dst = Y + (int64_t)m * ldy + nb;
-            if (vec_ok && nb + 8 <= N) {
-              *reinterpret_cast<uint4*>(dst) = v;
-            } else {
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-              for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
-            }
-          }
-        }
-        __syncwarp();
-      }
+      store_tile(tmem, warp, lane, scale, stage, Y, ldy, M, N, mt * kBN, nt * kBM);
       // every TMEM read of this tile has completed (tcgen05.wait::ld above)
       ptx::tc_fence_before();
       __syncwarp();
@@ -343,12 +419,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   - warp 0 of each CTA: TMA of its own stage bytes (codes and scale atoms)
 //     into its own shared memory, all counted on the even CTA's `full`
 //     (the odd CTA's loads use the pair form of the tensor copy);
+//   - warps 18..20 of the even CTA: the scale-factor copies (pair form), one
+//     warp per atom as in the one-SM kernel, committed to "sf_full";
 //   - warp 1 of the even CTA: the MMA issuer; its commits arrive on both
 //     CTAs' barriers;
-//   - warps 2..5: the epilogue of each CTA's accumulator rows; the even
-//     CTA's issuer waits for both epilogues (acc_empty, 8 arrivals) before it
-//     overwrites the accumulator.
+//   - warps 2..17: the epilogue of each CTA's accumulator rows; the even
+//     CTA's issuer waits for both epilogues (acc_empty, 32 arrivals) before
+//     it overwrites the accumulator.
 constexpr int kPairStages = 5;
+constexpr int kPairThreads = kThreads;                 // the same warp roles
 constexpr int kPairBBytes = (kBN / 2) * 128;          // this CTA's 128 tokens of a stage
 constexpr int kPairStageBytes = kABytes + kPairBBytes + kSFABytes + kSFBBytes;
 constexpr uint32_t kPairIdesc = ptx::idesc_nvf4(2 * kBM, kBN);
@@ -358,6 +437,8 @@ static_assert(kSfCol0 + kPairStages * 4 * kSfColsPerMma <= kTmemCols, "TMEM colu
 struct PairBars {
   uint64_t full[kPairStages];       // (even CTA) both CTAs' bytes of the stage have landed
   uint64_t empty[kPairStages];      // the pair's MMAs that read the stage are done
+  uint64_t sf_full[kPairStages];    // the stage's scale factors are in both CTAs' tensor memory
+  uint64_t sf_done;                 // (even CTA) every scale-factor copy has finished (teardown)
   uint64_t acc_full;                // the tile's accumulator is complete
   uint64_t acc_empty;               // (even CTA) both CTAs' epilogues have read it
   uint64_t mma_done;                // every MMA of the pair has finished (teardown)
@@ -381,7 +462,7 @@ __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, PairBa
 // Persistent pairs: cluster c = blockIdx.x / 2 takes the pair tiles
 // t = c, c + gridDim.x / 2, ... (weight rows 256 (t % tiles_n), tokens
 // 256 (t / tiles_n)); both CTAs walk the same tiles and stages.
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     gemm_w4a4_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                           const __grid_constant__ CUtensorMap tmap_sa, const __grid_constant__ CUtensorMap tmap_sb,
                           const float* __restrict__ g, const float* __restrict__ x_amax, uint16_t* __restrict__ Y,
@@ -409,7 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int st = 0; st < kPairStages; ++st) {
       ptx::mbar_init(&bars->full[st], 1);
       ptx::mbar_init(&bars->empty[st], 1);
+      ptx::mbar_init(&bars->sf_full[st], kSfWarps);
     }
+    ptx::mbar_init(&bars->sf_done, kSfWarps);
     ptx::mbar_init(&bars->acc_full, 1);
     ptx::mbar_init(&bars->acc_empty, 2 * kEpiWarps);
     ptx::mbar_init(&bars->mma_done, 1);
@@ -514,19 +597,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < num_ks; ++ks, ++gi) {
             const int st = gi % kPairStages;
             const uint32_t par = (uint32_t)(gi / kPairStages) & 1u;
-            if (!pair_wait(&bars->full[st], par, bars)) {
+            if (!pair_wait(&bars->full[st], par, bars) || !pair_wait(&bars->sf_full[st], par, bars)) {
               ok = false;
               break;
             }
             ptx::tc_fence_after();
             const uint32_t a0 = ptx::smem_u32(a_tile(st)), b0 = ptx::smem_u32(b_tile(st));
-            const uint32_t fa = ptx::smem_u32(sfa(st)), fb = ptx::smem_u32(sfb(st));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma;
-              ptx::tmem_copy_sf_pair(col, ptx::rows16_desc(fa + kk * 512));
-              ptx::tmem_copy_sf_pair(col + 4, ptx::rows16_desc(fb + kk * 512));
-              ptx::tmem_copy_sf_pair(col + 8, ptx::rows16_desc(fb + 2048 + kk * 512));
               ptx::mma_nvf4_pair(tmem, ptx::sw128_kmajor_desc(a0 + 32 * kk), ptx::sw128_kmajor_desc(b0 + 32 * kk),
                                  kPairIdesc, col, col + 4, (ks | kk) != 0);
             }
@@ -541,48 +620,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::mbar_wait_cluster(&bars->mma_done, 0, kWaitLimitNs);
     }
+  } else if (warp >= kSfWarp0) {
+    // ------------------ scale factors into both CTAs' tensor memory (even CTA)
+    // copy warp j: atom j of each MMA, as in the one-SM kernel, with the pair
+    // form of tcgen05.cp (each CTA's atom from its own shared memory)
+    const uint32_t j = (uint32_t)(warp - kSfWarp0);
+    if (lane == 0 && rank == 0) {
+      int gi = 0;
+      bool ok = true;
+      for (int t = cluster; t < tiles && ok; t += clusters) {
+        for (int ks = 0; ks < num_ks; ++ks, ++gi) {
+          const int st = gi % kPairStages;
+          if (!pair_wait(&bars->full[st], (uint32_t)(gi / kPairStages) & 1u, bars)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t src = j == 0 ? ptx::smem_u32(sfa(st)) : ptx::smem_u32(sfb(st)) + 2048u * (j - 1);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t col = tmem + kSfCol0 + (uint32_t)(st * 4 + kk) * kSfColsPerMma + 4u * j;
+            ptx::tmem_copy_sf_pair(col, ptx::rows16_desc(src + kk * 512));
+          }
+          ptx::mma_commit_pair(&bars->sf_full[st]);
+        }
+      }
+      // every copy done before the cluster's teardown (also on the error path)
+      ptx::mma_commit_pair(&bars->sf_done);
+      ptx::mbar_wait_cluster(&bars->sf_done, 0, kWaitLimitNs);
+    }
   } else {
     // ----------------------------------------------------------------- epilogue
     asm volatile("griddepcontrol.wait;" ::: "memory");  // x_amax and Y
-    const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. +31 = this CTA's weight rows
     const float scale = __fmul_rn(*g, __fdiv_rn(*x_amax, 2688.0f));
-    const uint32_t stage = ptx::smem_u32(epi) + (uint32_t)(warp - kEpiWarp0) * 2048u;
-    const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+    const uint32_t stage = ptx::smem_u32(epi) + (uint32_t)(warp - kEpiWarp0) * 512u;
     int it = 0;
     for (int t = cluster; t < tiles; t += clusters, ++it) {
       const int nt = t % tiles_n, mt = t / tiles_n;
-      const int n0 = nt * 2 * kBM + (int)rank * kBM, m0 = mt * kBN;
       if (!__all_sync(0xFFFFFFFFu, pair_wait(&bars->acc_full, it & 1, bars))) break;
       ptx::tc_fence_after();
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBN && m0 + c0 < M; c0 += 32) {
-        uint32_t rr[32];
-        ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
-        ptx::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(rr[j]) * scale);
-          st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
-        }
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
-          const int m = m0 + c0 + j;
-          const int nb = n0 + 32 * quarter + 8 * piece;
-          if (m < M && nb < N) {
-            const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
-            uint16_t* dst = Y + (int64_t)m * ldy + nb;
-            if (vec_ok && nb + 8 <= N) {
-              *reinterpret_cast<uint4*>(dst) = v;
-            } else {
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-              for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
-            }
-          }
-        }
-        __syncwarp();
-      }
+      // this CTA's accumulator rows are weight rows nt * 256 + 128 * rank + lane
+      store_tile(tmem, warp, lane, scale, stage, Y, ldy, M, N, mt * kBN, nt * 2 * kBM + (int)rank * kBM);
       // every TMEM read of this tile has completed (tcgen05.wait::ld above)
       ptx::tc_fence_before();
       __syncwarp();
@@ -764,7 +842,7 @@ cudaError_t launch_gemm_w4a4(const uint8_t* qx, const uint8_t* sx, const float* 
     const int64_t clusters = tiles < sms / 2 ? tiles : sms / 2;  // one persistent pair per two SMs at most
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * clusters));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kPairThreads);
     cfg.dynamicSmemBytes = kPairSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
