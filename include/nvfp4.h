@@ -105,8 +105,8 @@ typedef enum nvfp4_status {
  * both): a token tile then crosses from L2 into the SMs once per 256 weight
  * rows instead of once per 128.  The result is the same as without the flag
  * (same products, same fp32 accumulation order per output).  On one B200 the
- * [17408, 5120] layer at M = 512 ran at 38.7 us per call with the flag and
- * 35.3 us without (each stage then waits for the later of two CTAs' loads),
+ * [17408, 5120] layer at M = 512 ran at 28.5 us per call with the flag and
+ * 27.8 us without (each stage then waits for the later of two CTAs' loads),
  * so it is off by default.
  */
 #define NVFP4_FLAG_W4A4_PAIR (1u << 12)
