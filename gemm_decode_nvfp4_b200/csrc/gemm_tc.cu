@@ -56,7 +56,8 @@ constexpr int kBM = 128;        // weight rows per tile (MMA M)
 constexpr int kBK = 64;         // k per stage: one 128-byte swizzle row of f16
 constexpr int kDeqWarp0 = 2;    // warps 2..9 dequantize, then run the epilogue
 constexpr int kDeqWarps = 8;
-constexpr int kThreads = (kDeqWarp0 + kDeqWarps) * 32;
+constexpr int kEpiWarps = 16;   // warps 2..17 run the epilogue (10..17 only that)
+constexpr int kThreads = (kDeqWarp0 + kEpiWarps) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kWideRow = -(1 << 30);  // row-info marker: recompute this row exactly
 
@@ -99,6 +100,7 @@ struct Cfg {
   static_assert(kWStages >= 2, "weight ring needs two stages");
   static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(kBNT <= 512, "TMEM has 512 columns");
+  static_assert(kEpiWarps * 2048 <= kStages * kABytes, "epilogue staging blocks fit in the A ring");
 };
 
 __device__ __forceinline__ bool wait_or_fail(uint64_t* bar, uint32_t parity, Bars* bars) {
@@ -423,6 +425,62 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (bars->err) ptx::mbar_wait(&bars->tmem_full, 0, kWaitLimitNs);
     }
   } else {
+    // Epilogue of warp `warp` (any of the kEpiWarps): TMEM lane
+    // (32 * (warp % 4) + lane) holds weight row n; columns are m.  The warps
+    // of a lane quarter split the columns (when there are enough); each
+    // 32 x 32 block goes through 2 KB of the (now idle) A ring, so that Y is
+    // written as 64-byte row segments with 16-byte stores.
+    auto epilogue = [&]() {
+      if (!__all_sync(0xFFFFFFFFu, wait_or_fail(&bars->tmem_full, 0, bars))) return;
+      ptx::tc_fence_after();
+      const int quarter = warp & 3;
+      const float gv = *g;
+      constexpr int kParts = BNT >= 128 ? kEpiWarps / 4 : (BNT >= 64 ? 2 : 1);
+      constexpr int kColsPerWarp = BNT / kParts;
+      const int part = (warp - kDeqWarp0) >> 2;
+      if (part >= kParts) return;
+      const int c_begin = part * kColsPerWarp;
+      const uint32_t stage = ptx::smem_u32(a_tile(0)) + (uint32_t)(warp - kDeqWarp0) * 2048u;
+      const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
+#pragma unroll 1
+      for (int c0 = c_begin; c0 < c_begin + kColsPerWarp; c0 += 32) {
+        uint32_t rr[32];
+        ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const __nv_bfloat16 o = __float2bfloat16_rn((__uint_as_float(rr[j]) * gv) * bars->colpow[c0 + j]);
+          st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
+        }
+        __syncwarp();
+        // row j of the block: 32 consecutive n = 64 bytes, four lanes per row
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
+          const int m = m0 + c0 + j;
+          const int nb = n0 + 32 * quarter + 8 * piece;
+          if (c0 + j < c_begin + kColsPerWarp && m < M && bars->info[c0 + j] != kWideRow && nb < N) {
+            const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
+            uint16_t* dst = Y + (int64_t)m * ldy + nb;
+            if (vec_ok && nb + 8 <= N) {
+              *reinterpret_cast<uint4*>(dst) = v;
+            } else {
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+              for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
+            }
+          }
+        }
+        __syncwarp();
+      }
+    };
+    if (warp >= kDeqWarp0 + kDeqWarps) {
+      // ------------------------------------------------ epilogue only
+      if (static_weights) asm volatile("griddepcontrol.wait;" ::: "memory");  // Y
+      // wait (in the barrier, not polling) until the dequantization warps have
+      // staged the tile's row info, after their last stage
+      group_any(1, kEpiWarps * 32, false);
+      epilogue();
+    } else {
     // ------------------------------------------------ dequantize, then epilogue
     const int t = threadIdx.x - kDeqWarp0 * 32;  // 0..255
     const int r = t >> 1, h = t & 1;              // weight row in the tile, half of each 64 k
@@ -473,57 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bars->colpow[i] = e == kWideRow ? 1.0f : pow2f(-e);
       wide_here |= e == kWideRow;
     }
-    const bool any_wide = group_any(1, kDeqWarps * 32, wide_here);
-    // epilogue: TMEM lane (32 * (warp % 4) + lane) holds weight row n; columns are m.
-    const bool acc_ready = __all_sync(0xFFFFFFFFu, wait_or_fail(&bars->tmem_full, 0, bars));
-    if (acc_ready) {
-      ptx::tc_fence_after();
-      const int quarter = warp & 3;
-      const int n = n0 + 32 * quarter + lane;
-      const float gv = *g;
-      // the two warps of a lane quarter split the columns (when there are enough)
-      const int half_id = (warp - kDeqWarp0) >> 2;  // 0 or 1
-      constexpr int kColsPerWarp = BNT >= 64 ? BNT / 2 : BNT;
-      const int c_begin = BNT >= 64 ? half_id * kColsPerWarp : 0;
-      const bool active = BNT >= 64 || half_id == 0;
-      if (active) {
-        // Each 32 x 32 block (weight rows n of this lane quarter, activation
-        // rows m) goes through a 2 KB staging area in the (now idle) A ring, so
-        // that Y is written as 64-byte row segments with 16-byte stores.
-        const uint32_t stage = ptx::smem_u32(a_tile(0)) + (uint32_t)(warp - kDeqWarp0) * 2048u;
-        const bool vec_ok = ((reinterpret_cast<uintptr_t>(Y) & 15u) == 0) && (ldy % 8 == 0);
-#pragma unroll 1
-        for (int c0 = c_begin; c0 < c_begin + kColsPerWarp; c0 += 32) {
-          uint32_t rr[32];
-          ptx::tmem_ld_32cols(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0, rr);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const __nv_bfloat16 o = __float2bfloat16_rn((__uint_as_float(rr[j]) * gv) * bars->colpow[c0 + j]);
-            st_shared_u16(stage + (uint32_t)(j * 32 + lane) * 2u, *reinterpret_cast<const uint16_t*>(&o));
-          }
-          __syncwarp();
-          // row j of the block: 32 consecutive n = 64 bytes, four lanes per row
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int p = 32 * k + lane, j = p >> 2, piece = p & 3;
-            const int m = m0 + c0 + j;
-            const int nb = n0 + 32 * quarter + 8 * piece;
-            if (c0 + j < c_begin + kColsPerWarp && m < M && bars->info[c0 + j] != kWideRow && nb < N) {
-              const uint4 v = ld_shared_v4(stage + (uint32_t)(j * 32 + 8 * piece) * 2u);
-              uint16_t* dst = Y + (int64_t)m * ldy + nb;
-              if (vec_ok && nb + 8 <= N) {
-                *reinterpret_cast<uint4*>(dst) = v;
-              } else {
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                for (int i = 0; i < 8 && nb + i < N; ++i) dst[i] = (uint16_t)(w4[i >> 1] >> (16 * (i & 1)));
-              }
-            }
-          }
-          __syncwarp();
-        }
-      }
-    }
+    const bool any_wide = group_any(1, kEpiWarps * 32, wide_here);
+    epilogue();
     // rows of X outside the exact f16 window: exact fp32 dot on CUDA cores,
     // two threads per weight row (halves of K), combined with one shuffle
     const float gv = *g;
@@ -538,6 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const __nv_bfloat16 o = __float2bfloat16_rn(part * gv);
         Y[(int64_t)m * ldy + row] = *reinterpret_cast<const uint16_t*>(&o);
       }
+    }
     }
   }
 
