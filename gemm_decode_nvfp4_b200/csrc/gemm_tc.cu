@@ -32,7 +32,8 @@
 //     f16 into the swizzled A tile of each MMA stage;
 //   - warp 1, one thread: tcgen05.mma into the TMEM accumulator [128, BNT],
 //     committing each stage to its "empty" barrier;
-//   - warps 2..9 then read TMEM, apply g * 2^-e_m and store BF16 Y.
+//   - warps 2..17 (the dequant warps and eight that wait for the last MMA in
+//     a named barrier) then read TMEM, apply g * 2^-e_m and store BF16 Y.
 // Kernels are launched with programmatic dependent launch: with static
 // weights the W tiles start streaming while the previous kernel (the X prep)
 // is still running; X', e_m and Y are touched only after it completes.
