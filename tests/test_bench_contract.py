@@ -3,6 +3,7 @@ is divided by, against the per-call figures worked out from the formats
 (nibbles, one E4M3 scale per 16 or one UE8M0 per 32, BF16 activations and
 outputs, one fp32 tensor scale), and the source lists that key the committed
 DRAM-traffic figures."""
+import json
 import os
 
 import bench
@@ -79,3 +80,19 @@ def test_moe_multi_token_bytes():
     P = bench.MOE_T * bench.MOE["top"]
     e = 1536 * 2048 // 2 + 1536 * 2048 // 16
     assert bench.moe_bytes(P, 1536, 2048) + 2 * 2048 * (bench.MOE_T - 1) == P * (e + 2 * 1536 + 8 + 4) + 2 * 2048 * bench.MOE_T
+
+
+def test_traffic_only_for_the_source_it_was_taken_on(tmp_path, monkeypatch):
+    # a committed DRAM figure is reported while the row's kernel sources are
+    # unchanged, and becomes None (reported as null) once any of them changes
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setitem(bench.KERNEL_SOURCES, "gemv", ["k.cu"])
+    table = {"gemv": {"dram_bytes_per_call": 123, "source_hash": bench.kernel_source_hash(["k.cu"])}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(table))
+    assert bench.traffic_from_profiles("gemv") == 123
+    src.write_text("kernel v2\n")
+    assert bench.traffic_from_profiles("gemv") is None
+    assert bench.traffic_from_profiles("gemm_m32") is None  # no entry for the row
